@@ -1,0 +1,144 @@
+"""Pins for the FP8 part of the oracle: the e4m3 format against torch's
+independent conversion, the Hadamard rotation by its algebra, block
+quantisation by its defining properties, and the emulated FP8 attention
+against exact attention within the error that e4m3 rounding allows."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synthetic import attention_inputs, bf16_bits_to_f32, sign_vector
+
+
+def test_e4m3_round_matches_torch_in_range():
+    rng = np.random.default_rng(0)
+    x = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.uniform(-4, 2.3, 20000),
+        np.linspace(-448, 448, 4001),
+    ]).astype(np.float32)
+    x = x[np.abs(x) <= 448]
+    ours = oracle.e4m3_round(x)
+    theirs = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float32).numpy()
+    np.testing.assert_array_equal(ours, theirs)
+
+
+def test_e4m3_ties_go_to_even_and_saturate():
+    # 17 lies halfway between 16 and 18 (quantum 2 in [16, 32)): even mantissa is 16
+    assert oracle.e4m3_round(np.float32(17.0)) == 16.0
+    assert oracle.e4m3_round(np.float32(19.0)) == 20.0
+    # subnormal quantum is 2^-9; 2^-10 is a tie between 0 and 2^-9
+    assert oracle.e4m3_round(np.float32(2.0 ** -10)) == 0.0
+    assert oracle.e4m3_round(np.float32(3 * 2.0 ** -10)) == 2.0 ** -8
+    for big in (449.0, 464.0, 470.0, 1e6):
+        assert oracle.e4m3_round(np.float32(big)) == 448.0
+        assert oracle.e4m3_round(np.float32(-big)) == -448.0
+
+
+def test_e4m3_codes_match_torch_bit_patterns():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    theirs = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = oracle.e4m3_decode(codes)
+    np.testing.assert_array_equal(ours, theirs)
+    back = oracle.e4m3_encode(ours)
+    same = (back == codes) | ((codes & 0x7F) == 0)   # +-0
+    assert np.all(same)
+    assert np.isnan(oracle.e4m3_decode(np.array([0x7F, 0xFF], np.uint8))).all()
+
+
+@pytest.mark.parametrize("d", [1, 2, 8, 64, 128])
+def test_hadamard_is_orthogonal_sylvester(d):
+    h = oracle.hadamard(d)
+    np.testing.assert_array_equal(h @ h.T, d * np.eye(d))
+    assert set(np.unique(h)) <= {-1.0, 1.0}
+    if d >= 2:
+        half = oracle.hadamard(d // 2)
+        np.testing.assert_array_equal(h[: d // 2, : d // 2], half)
+        np.testing.assert_array_equal(h[d // 2:, d // 2:], -half)
+
+
+def test_rotation_preserves_scores_up_to_d():
+    rng = np.random.default_rng(1)
+    d = 128
+    q, k = rng.standard_normal((40, d)), rng.standard_normal((50, d))
+    sigma = sign_vector(7, d)
+    qr, kr = oracle.rotate_rows(q, sigma), oracle.rotate_rows(k, sigma)
+    np.testing.assert_allclose(qr @ kr.T, d * (q @ k.T), rtol=1e-12, atol=1e-12)
+    # a different sign vector for K breaks it
+    kbad = oracle.rotate_rows(k, sign_vector(8, d))
+    assert np.max(np.abs(qr @ kbad.T - d * (q @ k.T))) > 1.0
+
+
+def test_block_quantize_properties():
+    rng = np.random.default_rng(2)
+    y = rng.standard_normal((2, 3, 150, 64)) * np.exp(rng.standard_normal((2, 3, 150, 1)))
+    vals, scales = oracle.block_quantize(y, 64)
+    assert scales.shape == (2, 3, 3)
+    y32 = y.astype(np.float32).astype(np.float64)
+    for bi in range(3):
+        blk = y32[..., bi * 64:(bi + 1) * 64, :]
+        amax = np.abs(blk).max(axis=(-2, -1))
+        np.testing.assert_allclose(scales[..., bi], amax / 448.0, rtol=2 ** -23)
+        q = vals[..., bi * 64:(bi + 1) * 64, :].astype(np.float64)
+        assert np.all(np.abs(q) <= 448)
+        assert np.all(np.abs(q).max(axis=(-2, -1)) == 448.0)   # the amax element maps to 448
+        err = np.abs(q * scales[..., bi, None, None] - blk)
+        # half a quantum: 2^-4 relative in the normal range, 2^-10 s below it
+        bound = np.maximum(np.abs(blk) * 2.0 ** -4, 2.0 ** -10 * scales[..., bi, None, None]) * (1 + 1e-6)
+        assert np.all(err <= bound)
+    # an all-zero block keeps scale 1
+    v0, s0 = oracle.block_quantize(np.zeros((1, 64, 8)), 64)
+    assert s0[0, 0] == 1.0 and np.all(v0 == 0)
+
+
+def _fp8_inputs(N=256, d=64, H=2, seed=11, outliers=0.001):
+    x = attention_inputs(1, H, H, N, d, seed=seed, outlier_rate=outliers, with_dout=False)
+    return [bf16_bits_to_f32(x[n]).astype(np.float64) for n in ("q", "k", "v")]
+
+
+@pytest.mark.parametrize("rotate", [False, True])
+def test_fp8_emulation_within_e4m3_error_of_exact(rotate):
+    q, k, v = _fp8_inputs()
+    d = q.shape[-1]
+    scale = d ** -0.5
+    exact, lse = oracle.attention_forward(q, k, v, False, scale)
+    sigma = sign_vector(5, d) if rotate else None
+    o8, lse8 = oracle.fp8_attention_forward(q, k, v, False, scale, sigma)
+    rel = np.linalg.norm(o8 - exact) / np.linalg.norm(exact)
+    assert rel < 0.08, rel
+    # per-element quantisation error of S is about 2^-4 relative: a few
+    # hundredths on average, a few tenths at worst over all rows
+    assert np.mean(np.abs(lse8 - lse)) < 0.05
+    assert np.max(np.abs(lse8 - lse)) < 0.5
+
+
+def test_fp8_emulation_exact_when_operands_on_grid():
+    """Q, K, V already on the e4m3 grid with block amax 448 quantise exactly;
+    the only remaining error is P's e4m3 rounding: at most 2^-4 relative per
+    term (plus the subnormal floor), so |O - O_exact| <= 2^-4 max|V| + small."""
+    rng = np.random.default_rng(3)
+    N, d = 128, 64
+    def grid(shape):
+        x = oracle.e4m3_round((rng.standard_normal(shape) * 40).astype(np.float32)).astype(np.float64)
+        x[..., ::64, 0] = 448.0   # every 64-row block has amax exactly 448
+        return x
+    q, k, v = grid((1, 1, N, d)), grid((1, 1, N, d)), grid((1, 1, N, d))
+    scale = 1.0 / 4096
+    exact, _ = oracle.attention_forward(q, k, v, False, scale)
+    o8, _ = oracle.fp8_attention_forward(q, k, v, False, scale, None)
+    assert np.max(np.abs(o8 - exact)) <= 2.0 ** -4 * 448 + 1e-9
+
+
+def test_naive_fp8_is_worse_with_outliers():
+    """Reported, not a pin of the 2.6x figure: with entry outliers, block
+    scales plus rotation should not be worse than one scale per tensor."""
+    q, k, v = _fp8_inputs(N=256, d=64, seed=12, outliers=0.01)
+    scale = 64 ** -0.5
+    exact, _ = oracle.attention_forward(q, k, v, False, scale)
+    o_blk, _ = oracle.fp8_attention_forward(q, k, v, False, scale, sign_vector(9, 64))
+    o_naive = oracle.naive_fp8_attention_forward(q, k, v, False, scale)
+    rmse = lambda a: math.sqrt(np.mean((a - exact) ** 2))
+    assert rmse(o_blk) < rmse(o_naive)
+    assert np.linalg.norm(o_naive - exact) / np.linalg.norm(exact) < 0.3
