@@ -1,0 +1,137 @@
+"""Same-named Python entry points over the C ABI (argument marshalling only)."""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _lib
+
+FA_OK = 0
+_STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_MISALIGNED",
+           4: "FA_ERR_WORKSPACE", 5: "FA_ERR_CUDA", 6: "FA_ERR_TIMEOUT"}
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} returned {fa_status_string(status)} ({status})")
+
+
+def fa_status_string(status: int) -> str:
+    return _lib.load().fa_status_string(int(status)).decode()
+
+
+def fa_last_device_status() -> int:
+    """Device status word (0 = no kernel gave up on a bounded wait); clears it."""
+    return int(_lib.load().fa_last_device_status())
+
+
+def fa_bwd_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
+    return int(_lib.load().fa_bwd_workspace_size(B, Hq, Hkv, N, d))
+
+
+def fa_fp8_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
+    return int(_lib.load().fa_fp8_workspace_size(B, Hq, Hkv, N, d))
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(name: str, t: torch.Tensor, dtype, shape) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _dims(q, k):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, H, N, d]")
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    return B, Hq, Hkv, N, d
+
+
+def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None):
+    """O, LSE = attention(q, k, v). q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 (CUDA);
+    returns O bf16 [B,Hq,N,d] and LSE float32 [B,Hq,N]."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    _check("q", q, torch.bfloat16, (B, Hq, N, d))
+    _check("k", k, torch.bfloat16, (B, Hkv, N, d))
+    _check("v", v, torch.bfloat16, (B, Hkv, N, d))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _check("out", out, torch.bfloat16, (B, Hq, N, d))
+    _check("lse", lse, torch.float32, (B, Hq, N))
+    st = _lib.load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                            B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    if st != FA_OK:
+        raise FAError("fa_fwd", st)
+    return out, lse
+
+
+def fa_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+           dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of attention(q, k, v) against dout, recomputing P from lse."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    for name, t, shp in (("q", q, (B, Hq, N, d)), ("k", k, (B, Hkv, N, d)), ("v", v, (B, Hkv, N, d)),
+                         ("o", o, (B, Hq, N, d)), ("dout", dout, (B, Hq, N, d))):
+        _check(name, t, torch.bfloat16, shp)
+    _check("lse", lse, torch.float32, (B, Hq, N))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check("dq", dq, torch.bfloat16, (B, Hq, N, d))
+    _check("dk", dk, torch.bfloat16, (B, Hkv, N, d))
+    _check("dv", dv, torch.bfloat16, (B, Hkv, N, d))
+    ws_bytes = fa_bwd_workspace_size(B, Hq, Hkv, N, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    st = _lib.load().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                            dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                            B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    if st != FA_OK:
+        raise FAError("fa_bwd", st)
+    return dq, dk, dv
+
+
+def fa_fwd_fp8(q, k, v, causal: bool = False, scale: float | None = None, rotation_seed: int = 0,
+               use_rotation: bool = True, out=None, lse=None, workspace=None, stream=None):
+    """FP8 (e4m3) forward with 64-row block scales and optional Hadamard
+    rotation of Q and K; bf16 inputs and output."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    _check("q", q, torch.bfloat16, (B, Hq, N, d))
+    _check("k", k, torch.bfloat16, (B, Hkv, N, d))
+    _check("v", v, torch.bfloat16, (B, Hkv, N, d))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    ws_bytes = fa_fp8_workspace_size(B, Hq, Hkv, N, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    st = _lib.load().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                int(rotation_seed) & 0xFFFFFFFFFFFFFFFF, int(bool(use_rotation)),
+                                workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    if st != FA_OK:
+        raise FAError("fa_fwd_fp8", st)
+    return out, lse

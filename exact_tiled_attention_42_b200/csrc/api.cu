@@ -1,0 +1,177 @@
+// The C ABI of include/fa.h: argument checks, TMA tensor maps, launches.
+//
+// Nothing here allocates device memory: every buffer, workspaces included,
+// belongs to the caller. The only host-side state is the driver entry point
+// for cuTensorMapEncodeTiled and the device address of the status word.
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+#include "kernels.h"
+
+namespace {
+
+__device__ int g_fa_status;  // first bounded-wait failure since it was last read
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+std::mutex g_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Device address of g_fa_status on the current device (looked up once).
+int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_shape(int B, int Hq, int Hkv, int N, int d, float scale) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(B) * Hq;
+  const long long tiles = (N + 127) / 128;
+  if (BH > 0x7fffffffLL || (tiles + 1) / 2 > 65535) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+// 3-D map over a [rows_outer, N, d] bf16 tensor: box of 64 columns x box_rows rows.
+bool make_map_bf16(CUtensorMap* m, const void* ptr, int d, int N, long long outer, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+int fa_last_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fa_status, sizeof(int)) != cudaSuccess) return -1;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_fa_status, &zero, sizeof(int)) != cudaSuccess) return -1;
+  return v;
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                 int d, int causal, float scale, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  fa_status st = check_shape(B, Hq, Hkv, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  CUtensorMap tmQ, tmK, tmV, tmO;
+  const long long BH = static_cast<long long>(B) * Hq, BHkv = static_cast<long long>(B) * Hkv;
+  if (!make_map_bf16(&tmQ, q, d, N, BH, 128) || !make_map_bf16(&tmK, k, d, N, BHkv, 128) ||
+      !make_map_bf16(&tmV, v, d, N, BHkv, 128) || !make_map_bf16(&tmO, o, d, N, BH, 128))
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.lse = lse;
+  p.status = status_ptr();
+  p.N = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.num_qtiles = (N + 127) / 128;
+  p.num_pairs = (p.num_qtiles + 1) / 2;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (!p.status) return FA_ERR_CUDA;
+  cudaError_t e = fa::launch_fwd_bf16(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), d, causal != 0, stream);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {
+  if (check_shape(B, Hq, Hkv, N, d, 1.0f) != FA_OK) return 0;
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t rows = static_cast<size_t>(B) * Hq * N;
+  return up(rows * sizeof(float)) + up(rows * d * sizeof(float));
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N,
+                 int d, int causal, float scale, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  fa_status st = check_shape(B, Hq, Hkv, N, d, scale);
+  if (st != FA_OK) return st;
+  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < fa_bwd_workspace_size(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  (void)causal;
+  (void)stream;
+  return FA_ERR_UNSUPPORTED;  // backward kernel not built yet
+}
+
+size_t fa_fp8_workspace_size(int B, int Hq, int Hkv, int N, int d) {
+  if (check_shape(B, Hq, Hkv, N, d, 1.0f) != FA_OK) return 0;
+  auto up = [](size_t x) { return (x + 1023) & ~static_cast<size_t>(1023); };
+  const size_t nb = (N + 63) / 64;
+  const size_t q = static_cast<size_t>(B) * Hq, kv = static_cast<size_t>(B) * Hkv;
+  return up(q * N * d) + 2 * up(kv * N * d) + up(q * nb * 4) + 2 * up(kv * nb * 4);
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, uint64_t rotation_seed,
+                     int use_rotation, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d,
+                     int causal, float scale, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  fa_status st = check_shape(B, Hq, Hkv, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < fa_fp8_workspace_size(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
+  (void)rotation_seed;
+  (void)use_rotation;
+  (void)causal;
+  (void)stream;
+  return FA_ERR_UNSUPPORTED;  // FP8 kernels not built yet
+}
+
+}  // extern "C"

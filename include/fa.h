@@ -1,0 +1,127 @@
+/*
+ * Exact tiled softmax attention for NVIDIA B200 (sm_100a): the C ABI.
+ *
+ * The operation. For every batch b and query head h, with kv = h / (Hq / Hkv):
+ *     S = scale * Q[b,h] K[b,kv]^T          (N x N, never written to memory)
+ *     S[i,j] = -inf  where causal and j > i
+ *     O[b,h] = softmax_rows(S) V[b,kv]
+ *     LSE[b,h,i] = log sum_j exp(S[i,j])    (natural log)
+ * "FlashAttention: The Algorithm That Made Long-Context AI Possible"
+ * (promptingindex.com), section "The quadratic bottleneck in standard
+ * attention", defines S = Q K^T and O = softmax(S) V; section "What tiling
+ * changes" gives the method: Q, K and V are split into blocks that fit on
+ * chip, a running row maximum and a running sum of exponentials make the
+ * softmax exact, and the N x N matrix never reaches high-bandwidth memory.
+ * "FlashAttention: Fast and Memory-Efficient Exact Attention with
+ * IO-Awareness" (abstract) states that the tiled algorithm is exact and needs
+ * linear, not quadratic, memory. The scale, the causal mask, the log-sum-exp
+ * output and the backward pass are not on those pages; they follow the
+ * workload statement the library is built to (scale = 1/sqrt(d) in every
+ * shipped workload, causal keeps j <= i).
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are DEVICE pointers unless said otherwise, 16-byte aligned.
+ *   - Tensors are row-major contiguous: Q, O, dO, dQ are [B, Hq, N, d];
+ *     K, V, dK, dV are [B, Hkv, N, d]; LSE and D are [B, Hq, N] float32.
+ *     bf16 tensors are passed as raw 16-bit storage.
+ *   - d is 64 or 128; N >= 1; Hq is a multiple of Hkv; scale is finite and > 0.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream), like a
+ *     kernel launch; outputs are valid once the stream has been synchronised.
+ *   - The caller owns every buffer, workspaces included. The library allocates
+ *     no device memory and keeps no state between calls.
+ *   - Every argument is checked before anything is launched; a failed check
+ *     returns an error and launches nothing. A launch error is returned as
+ *     FA_ERR_CUDA.
+ *   - Not safe to call concurrently on overlapping output buffers.
+ */
+#ifndef EXACT_TILED_ATTENTION_FA_H
+#define EXACT_TILED_ATTENTION_FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, Hq % Hkv != 0, bad scale */
+  FA_ERR_UNSUPPORTED = 2,  /* head dimension other than 64 / 128, or a size past the limits */
+  FA_ERR_MISALIGNED = 3,   /* a pointer that is not 16-byte aligned */
+  FA_ERR_WORKSPACE = 4,    /* workspace pointer null or smaller than the *_workspace_size query */
+  FA_ERR_CUDA = 5,         /* the CUDA runtime reported an error when launching */
+  FA_ERR_TIMEOUT = 6       /* a kernel gave up on a bounded wait (see fa_last_device_status) */
+} fa_status;
+
+/*
+ * Forward pass. Writes O (bf16, [B,Hq,N,d]) and LSE (float32, [B,Hq,N],
+ * natural log). `lse` may not be null (the backward needs it).
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                 cudaStream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) (float32,
+ * [B,Hq,N]) and the float32 dQ accumulator ([B,Hq,N,d]), each rounded up to
+ * 256 bytes. Linear in N. Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * Backward pass by recomputation: P is rebuilt from Q, K and the saved LSE,
+ * then dV = P^T dO, dP = dO V^T, dS = P * (dP - D), dQ = scale dS K,
+ * dK = scale dS^T Q, with dK and dV summed over the Hq / Hkv query heads that
+ * share a KV head. `o` and `lse` are fa_fwd's outputs for the same inputs.
+ * dq, dk, dv (bf16) are overwritten, not accumulated. The workspace is
+ * overwritten; its contents on entry do not matter.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv,
+                 void* workspace, size_t workspace_bytes,
+                 int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                 cudaStream_t stream);
+
+/*
+ * Bytes of device workspace fa_fwd_fp8 needs: e4m3 copies of Q, K, V
+ * (rotated Q and K) and one float32 scale per 64-row block of each. Returns 0
+ * for invalid sizes.
+ */
+size_t fa_fp8_workspace_size(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * FP8 (e4m3) forward with block quantisation and incoherent processing:
+ * "FlashAttention-3: Fast and Accurate Attention with Asynchrony and
+ * Low-precision" (abstract) names both techniques and gives neither the
+ * block shape nor the rotation. Here: Q and K are rotated by
+ * diag(sigma) H_d (Sylvester Hadamard, sigma a +-1 vector drawn from
+ * `rotation_seed` by SplitMix64, the same for Q and K) when use_rotation is
+ * non-zero; Q, K, V are quantised with one float32 scale per 64-row block
+ * (s = amax / 448); P is quantised per 128-key tile with V's block scale
+ * folded in. Inputs are bf16; O is bf16, LSE float32. The workspace is
+ * overwritten.
+ */
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                     uint64_t rotation_seed, int use_rotation,
+                     void* workspace, size_t workspace_bytes,
+                     int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                     cudaStream_t stream);
+
+/* Human-readable name of a status code (static storage, never null). */
+const char* fa_status_string(fa_status s);
+
+/*
+ * Device status word of the current device, then cleared. 0 when no kernel
+ * has given up on a bounded wait since the last call. Otherwise the low byte
+ * is an fa_status (FA_ERR_TIMEOUT) and bits 8.. name the wait that gave up.
+ * Synchronises the device. Returns -1 if the word could not be read.
+ */
+int fa_last_device_status(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_TILED_ATTENTION_FA_H */

@@ -1,0 +1,112 @@
+"""The C-ABI library: it loads, exports every symbol include/fa.h declares,
+and rejects bad arguments on the host before launching anything (no GPU
+needed for any of these)."""
+
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_tiled_attention_42_b200 import _lib
+    if not os.path.exists(_lib.LIB_PATH):
+        from exact_tiled_attention_42_b200.build import build
+        build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:fa_status|size_t|const char\*|int)\s+(fa_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for need in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_fwd_fp8", "fa_fp8_workspace_size",
+                 "fa_status_string", "fa_last_device_status"):
+        assert need in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(lib._name)
+    for name in declared_functions():
+        assert hasattr(raw, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    from exact_tiled_attention_42_b200 import _lib
+    assert set(declared_functions()) <= set(_lib.SIGNATURES)
+
+
+def test_status_strings(lib):
+    assert lib.fa_status_string(0) == b"FA_OK"
+    assert lib.fa_status_string(6) == b"FA_ERR_TIMEOUT"
+    assert lib.fa_status_string(99) == b"FA_ERR_UNKNOWN"
+
+
+P = 0x100000   # an aligned fake device address; never dereferenced by these calls
+
+
+def fwd(lib, q=P, k=P, v=P, o=P, lse=P, B=1, Hq=2, Hkv=2, N=128, d=64, causal=0, scale=0.125):
+    return lib.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, None)
+
+
+def test_fwd_rejects_bad_arguments(lib):
+    assert fwd(lib, q=None) == 1
+    assert fwd(lib, lse=None) == 1
+    assert fwd(lib, N=0) == 1
+    assert fwd(lib, B=0) == 1
+    assert fwd(lib, Hq=3, Hkv=2) == 1
+    assert fwd(lib, scale=0.0) == 1
+    assert fwd(lib, scale=-1.0) == 1
+    assert fwd(lib, scale=float("inf")) == 1
+    assert fwd(lib, scale=float("nan")) == 1
+    assert fwd(lib, d=96) == 2
+    assert fwd(lib, d=256) == 2
+    assert fwd(lib, N=65535 * 256 + 1) == 2
+    assert fwd(lib, q=P + 8) == 3
+    assert fwd(lib, lse=P + 4) == 3
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    ws = lib.fa_bwd_workspace_size(1, 2, 2, 128, 64)
+    def bwd(ws_ptr=P, ws_bytes=ws, d=64, dq=P):
+        return lib.fa_bwd(P, P, P, P, P, P, dq, P, P, ws_ptr, ws_bytes, 1, 2, 2, 128, d, 0, 0.125, None)
+    assert bwd(dq=None) == 1
+    assert bwd(d=80) == 2
+    assert bwd(ws_ptr=None) == 4
+    assert bwd(ws_bytes=ws - 1) == 4
+    assert bwd(dq=P + 2) == 3
+
+
+def test_fp8_rejects_bad_arguments(lib):
+    ws = lib.fa_fp8_workspace_size(1, 2, 2, 128, 128)
+    assert ws > 0
+    assert lib.fa_fwd_fp8(P, P, P, P, P, 1, 1, None, ws, 1, 2, 2, 128, 128, 0, 0.1, None) == 4
+    assert lib.fa_fwd_fp8(P, P, P, P, P, 1, 1, P, ws - 1, 1, 2, 2, 128, 128, 0, 0.1, None) == 4
+    assert lib.fa_fwd_fp8(P, P, None, P, P, 1, 1, P, ws, 1, 2, 2, 128, 128, 0, 0.1, None) == 1
+
+
+def test_workspace_sizes_are_linear_in_n(lib):
+    """The score matrix the pages size (4,096 tokens -> 16.7 million entries,
+    128K -> 16.4 billion) is never stored: workspace grows linearly in N."""
+    cases = json.load(open(os.path.join(ROOT, "tests", "golden", "score_matrix_sizes.json")))["cases"]
+    for c in cases:
+        n = c["tokens"]
+        assert abs(n * n - c["entries"]) <= c["rel_tol"] * c["entries"]
+        ws = lib.fa_bwd_workspace_size(1, 1, 1, n, 128)
+        assert ws < 4 * n * n / 8, (n, ws)
+    a = lib.fa_bwd_workspace_size(2, 8, 2, 4096, 128)
+    b = lib.fa_bwd_workspace_size(2, 8, 2, 8192, 128)
+    assert abs(b / a - 2.0) < 1e-3
+    assert lib.fa_bwd_workspace_size(1, 3, 2, 128, 64) == 0
+    f1 = lib.fa_fp8_workspace_size(1, 4, 4, 4096, 128)
+    f2 = lib.fa_fp8_workspace_size(1, 4, 4, 8192, 128)
+    assert abs(f2 / f1 - 2.0) < 1e-2
