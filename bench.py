@@ -51,15 +51,6 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def step_flops(w, passes=PASSES):
-    f = 0.0
-    if "fwd" in passes:
-        f += w.fwd_flops(CAUSAL)
-    if "bwd" in passes:
-        f += w.bwd_flops(CAUSAL)
-    return f
-
-
 class ClockSampler:
     """nvidia-smi clock/throttle samples during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -108,57 +99,89 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_oracle_sample(w, seconds_budget=15.0):
-    """Time the fp64 oracle on whole heads of the workload (head 0 of batch 0
-    first, then further heads) until the budget is spent; returns
-    (TFLOP/s, flops done, seconds, heads)."""
-    import oracle
+def _oracle_threads():
     try:
         import threadpoolctl
-        threads = max(v["num_threads"] for v in threadpoolctl.threadpool_info()) if threadpoolctl.threadpool_info() else os.cpu_count()
+        info = threadpoolctl.threadpool_info()
+        return max(v["num_threads"] for v in info) if info else os.cpu_count()
     except Exception:
-        threads = os.cpu_count()
+        return os.cpu_count()
+
+
+def _oracle_inputs(w):
     bits = attention_inputs(1, 1, 1, w.N, w.d, w.seed, with_dout=True)
-    x = {n: bf16_bits_to_f32(a).astype(np.float64) for n, a in bits.items()}
-    per_head = step_flops(w) / (w.B * w.Hq)
+    return {n: bf16_bits_to_f32(a).astype(np.float64) for n, a in bits.items()}
+
+
+def _oracle_rows(x, w, causal, passes, rows):
+    """One oracle sample: query rows ``rows`` of one (batch, head) problem."""
+    import oracle
+    oracle.attention_forward(x["q"], x["k"], x["v"], causal, w.scale, rows=rows)
+    if "bwd" in passes:
+        oracle.attention_backward(x["q"], x["k"], x["v"], x["do"], causal, w.scale, rows=rows)
+
+
+def _sample_flops(w, causal, passes, nrows):
+    """The workload's FLOP formula, per (batch, head), scaled to nrows rows."""
+    per_head = sum((w.fwd_flops(causal) if p_ == "fwd" else w.bwd_flops(causal)) for p_ in passes) / (w.B * w.Hq)
+    return per_head * nrows / w.N
+
+
+def cpu_oracle_sample(w, causal, passes, seconds_budget=15.0):
+    """Time the fp64 oracle on whole (batch, head) problems of the workload
+    until the budget is spent; returns (TFLOP/s, seconds, problems, threads)."""
+    x = _oracle_inputs(w)
     done, heads, t0 = 0.0, 0, time.perf_counter()
     while True:
-        oracle.attention_forward(x["q"], x["k"], x["v"], CAUSAL, w.scale)
-        if "bwd" in PASSES:
-            oracle.attention_backward(x["q"], x["k"], x["v"], x["do"], CAUSAL, w.scale)
+        _oracle_rows(x, w, causal, passes, None)
         heads += 1
-        done += per_head
+        done += _sample_flops(w, causal, passes, w.N)
         el = time.perf_counter() - t0
         if el > seconds_budget or heads >= 64:
             break
-    return done / el / 1e12, done, el, heads, threads
+    return done / el / 1e12, el, heads, _oracle_threads()
 
 
 def run_reference(args, rank, world):
+    """The oracle as it stands, on the host cores: each step is a block of
+    query rows around the middle of one (batch, head) problem (under a causal
+    mask their cost is the average row's), sized so that the K steps take
+    about a minute in total."""
     if rank != 0:
         return
-    w = WORKLOADS[WORKLOAD]
+    w = WORKLOADS[args.workload]
+    causal = w.causal[0]
+    passes = PASSES
+    x = _oracle_inputs(w)
+    # warm-up samples also calibrate the seconds per row
+    r_cal = min(64, w.N)
+    mid = w.N // 2
+    t_row = None
     for _ in range(args.warmup):
-        pass  # the oracle has no warm-up state; steps below are all timed
-    vals = []
-    t_all = 0.0
-    heads_all = 0
-    threads = os.cpu_count()
-    budget = max(2.0, 60.0 / max(1, args.steps))
+        t0 = time.perf_counter()
+        _oracle_rows(x, w, causal, passes, (mid - r_cal // 2, mid - r_cal // 2 + r_cal))
+        t_row = (time.perf_counter() - t0) / r_cal
+    per_step = max(0.05, 60.0 / max(1, args.steps))
+    nrows = int(max(1, min(w.N, per_step / max(t_row, 1e-9))))
+    r0 = max(0, mid - nrows // 2)
+    rows = (r0, r0 + nrows)
+    times = []
     for _ in range(args.steps):
-        v, _, el, heads, threads = cpu_oracle_sample(w, seconds_budget=budget)
-        vals.append(v)
-        t_all += el
-        heads_all += heads
-    value = statistics.median(vals)
+        t0 = time.perf_counter()
+        _oracle_rows(x, w, causal, passes, rows)
+        times.append(time.perf_counter() - t0)
+    t_step = statistics.mean(times)
+    value = _sample_flops(w, causal, passes, nrows) / t_step / 1e12
+    threads = _oracle_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_all / args.steps,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} causal={CAUSAL}",
-                   "passes": list(PASSES), "l2": "inputs larger than L2"},
+        "config": {"workload": f"{args.workload}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} causal={causal}",
+                   "passes": list(passes), "l2": "inputs larger than L2 (no flush between steps)"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{heads_all} whole (batch, head) problems of the workload over {args.steps} steps"},
+                         "sample": f"per step: query rows {rows[0]}..{rows[1] - 1} of one (batch, head) problem, "
+                                   f"fp64 numpy oracle, {len(passes)} pass(es)"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -172,8 +195,10 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     _lib.load()
-    w = WORKLOADS[WORKLOAD]
-    bits = attention_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, with_dout=("bwd" in PASSES))
+    w = WORKLOADS[args.workload]
+    causal = w.causal[0]
+    passes = PASSES
+    bits = attention_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, with_dout=("bwd" in passes))
     host = {n: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for n, a in bits.items()}
     dev = {n: t.cuda() for n, t in host.items()}
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
@@ -181,29 +206,31 @@ def run_ours(args, rank, world, local_rank):
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step():
-        fa.fa_fwd(dev["q"], dev["k"], dev["v"], causal=CAUSAL, out=o, lse=lse)
+    def fwd():
+        fa.fa_fwd(dev["q"], dev["k"], dev["v"], causal=causal, out=o, lse=lse)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     for _ in range(args.warmup):
-        step()
+        fwd()
     torch.cuda.synchronize()
     assert fa.fa_last_device_status() == 0
 
-    # --- device-timed region: K steps, per-launch events for the forward kernel
+    # --- device-timed region: K steps; events around each pass on the
+    # launching stream give the per-launch duration of each kernel
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
+        time.sleep(0.5)  # let nvidia-smi start sampling before the timed region
         t_start.record(stream)
         for i in range(args.steps):
             ev[i][0].record(stream)
-            step()
+            fwd()
             ev[i][1].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -215,58 +242,64 @@ def run_ours(args, rank, world, local_rank):
         t = torch.tensor([ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    flops = step_flops(w)
+    flops = sum((w.fwd_flops(causal) if p_ == "fwd" else w.bwd_flops(causal)) for p_ in passes)
     value = world * flops * args.steps / (ms * 1e-3) / 1e12
 
-    # --- end to end through the public API with pinned host buffers
-    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    h2d = sum(host[n].numel() * 2 for n in ("q", "k", "v"))
-    d2h = o_host.numel() * 2 + lse_host.numel() * 4
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        for n in ("q", "k", "v"):
-            dev[n].copy_(host[n], non_blocking=True)
-        step()
-        o_host.copy_(o, non_blocking=True)
-        lse_host.copy_(lse, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops * args.steps / (e2e_ms * 1e-3) / 1e12
+    # --- end to end through the public API with pinned host buffers: every
+    # step copies its inputs host->device and reads O and LSE back
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = min(args.steps, 50)
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h2d = sum(host[n].numel() * 2 for n in ("q", "k", "v"))
+        d2h = o_host.numel() * 2 + lse_host.numel() * 4
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            for n in ("q", "k", "v"):
+                dev[n].copy_(host[n], non_blocking=True)
+            fwd()
+            o_host.copy_(o, non_blocking=True)
+            lse_host.copy_(lse, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+    assert fa.fa_last_device_status() == 0
 
     if rank != 0:
         return
     pk, pk_kind = peaks()
     peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
     avg_fwd_ms = statistics.mean(fwd_ms)
-    achieved = w.fwd_flops(CAUSAL) / (avg_fwd_ms * 1e-3) / 1e12
+    achieved = w.fwd_flops(causal) / (avg_fwd_ms * 1e-3) / 1e12
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        v, done, el, heads, threads = cpu_oracle_sample(w, seconds_budget=args.cpu_seconds)
+        v, el, heads, threads = cpu_oracle_sample(w, causal, passes, seconds_budget=args.cpu_seconds)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{heads} whole (batch, head) problem(s) of the workload, fp64 numpy, {el:.1f} s"}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} causal={CAUSAL}",
-                   "passes": list(PASSES), "l2": "inputs larger than L2 (192 MiB of Q/K/V), no flush",
+        "config": {"workload": f"{args.workload}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} causal={causal}",
+                   "passes": list(passes), "l2": "inputs larger than L2 (no flush between steps)",
                    "parallelism": f"replica x{world} (independent problems per GPU)"},
         "fwd_tflops": achieved, "fwd_frac_of_peak": achieved / peak,
         "roofline": {"bound": "tensor", "kernel": "fwd_bf16_kernel", "achieved": achieved, "peak": peak,
-                     "peak_kind": f"{pk_kind} bf16 dense, sustained", "unit": "TFLOP/s", "frac": achieved / peak,
-                     "traffic": None},
+                     "peak_kind": f"{pk_kind} bf16 dense, sustained (kernel timed inside a long loop)",
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None},
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * len(PASSES),
+        "e2e": e2e,
+        "gpu_launches": args.steps * len(passes),
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
@@ -275,11 +308,14 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS),
+                    help="workload to run (profiling of other shapes; the headline is the default)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

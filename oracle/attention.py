@@ -74,37 +74,42 @@ def attention_probabilities(q, k, causal: bool, scale: float) -> np.ndarray:
     return p
 
 
-def attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int = 2048):
+def attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int = 2048, rows=None):
     """O = softmax(scale * Q K^T [+ causal mask]) V and LSE, in float64.
 
     Rows of S are formed ``row_chunk`` at a time so that large N fits in host
     memory; every row still sees its full set of scores, so this is the plain
-    definition, not a tiling of the key dimension.
+    definition, not a tiling of the key dimension. ``rows = (r0, r1)`` limits
+    the work to query rows r0..r1-1 (other rows of the result are left as
+    NaN); it changes which rows are computed, not how.
     Returns (O [B,Hq,N,d], LSE [B,Hq,N]).
     """
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
     B, Hq, Hkv, N, d, g = _heads(q, k)
-    o = np.empty((B, Hq, N, d))
-    lse = np.empty((B, Hq, N))
+    lo, hi = (0, N) if rows is None else rows
+    o = np.full((B, Hq, N, d), np.nan)
+    lse = np.full((B, Hq, N), np.nan)
     for b in range(B):
         for h in range(Hq):
             kh, vh = k[b, h // g], v[b, h // g]
-            for r0 in range(0, N, row_chunk):
-                r1 = min(N, r0 + row_chunk)
+            for r0 in range(lo, hi, row_chunk):
+                r1 = min(hi, r0 + row_chunk)
                 p, lse[b, h, r0:r1] = _softmax_rows(_scores(q[b, h], kh, scale, causal, r0, r1))
                 o[b, h, r0:r1] = p @ vh
     return o, lse
 
 
-def attention_backward(q, k, v, dout, causal: bool, scale: float, row_chunk: int = 2048):
+def attention_backward(q, k, v, dout, causal: bool, scale: float, row_chunk: int = 2048, rows=None):
     """Analytic gradients (dQ, dK, dV) of O = attention(Q, K, V) against dO.
 
     With P the softmax matrix:  dV = P^T dO;  dP = dO V^T;
     D_i = sum_t dO[i,t] O[i,t];  dS = P * (dP - D);  dQ = scale dS K;
     dK = scale dS^T Q.  dK and dV are summed over the query heads that share
     a KV head. P and O are recomputed here from the definition.
+    ``rows = (r0, r1)`` keeps only the terms of query rows r0..r1-1 (their dQ
+    rows and their share of dK and dV).
     """
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
@@ -114,12 +119,13 @@ def attention_backward(q, k, v, dout, causal: bool, scale: float, row_chunk: int
     dq = np.zeros((B, Hq, N, d))
     dk = np.zeros((B, Hkv, N, d))
     dv = np.zeros((B, Hkv, N, d))
+    lo, hi = (0, N) if rows is None else rows
     for b in range(B):
         for h in range(Hq):
             kv = h // g
             kh, vh = k[b, kv], v[b, kv]
-            for r0 in range(0, N, row_chunk):
-                r1 = min(N, r0 + row_chunk)
+            for r0 in range(lo, hi, row_chunk):
+                r1 = min(hi, r0 + row_chunk)
                 p, _ = _softmax_rows(_scores(q[b, h], kh, scale, causal, r0, r1))
                 do = dout[b, h, r0:r1]
                 o = p @ vh

@@ -185,6 +185,19 @@ def test_gqa_equals_repeated_heads():
         np.testing.assert_allclose(dv1, dv2.reshape(B, Hkv, grp, N, d).sum(2), atol=1e-13)
 
 
+def test_row_subset_matches_full_result():
+    q, k, v, do = (_rand((1, 2, 50, 8), s) for s in (24, 25, 26, 27))
+    full = oracle.attention_forward(q, k, v, True, 0.3)
+    part = oracle.attention_forward(q, k, v, True, 0.3, row_chunk=4, rows=(13, 31))
+    np.testing.assert_array_equal(part[0][:, :, 13:31], full[0][:, :, 13:31])
+    assert np.isnan(part[0][:, :, :13]).all() and np.isnan(part[1][:, :, 31:]).all()
+    g_full = oracle.attention_backward(q, k, v, do, True, 0.3)
+    g_a = oracle.attention_backward(q, k, v, do, True, 0.3, rows=(0, 20))
+    g_b = oracle.attention_backward(q, k, v, do, True, 0.3, rows=(20, 50))
+    for x, a, b in zip(g_full, g_a, g_b):
+        np.testing.assert_allclose(a + b, x, atol=1e-13)
+
+
 def test_row_chunking_does_not_change_result():
     q, k, v, do = (_rand((1, 2, 50, 8), s) for s in (20, 21, 22, 23))
     a = oracle.attention_forward(q, k, v, True, 0.3, row_chunk=7)
