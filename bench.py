@@ -4,7 +4,7 @@
 
 One step is one pass of the hot path over the long-sequence head-dim-128
 workload (B=2, Hq=Hkv=16, N=8192, d=128, causal, bf16 inputs drawn i.i.d.
-N(0,1)): the forward (O and LSE) and, once built, the recompute backward.
+N(0,1)): the forward (O and LSE) and the recompute backward (dQ, dK, dV).
 FLOPs follow the workload statement: 4*B*Hq*N^2*d for the forward, halved for
 the causal mask, and 2.5x that for the backward. Inputs (3 x 64 MiB) are
 larger than the 126 MB L2, so no flush runs between steps.
@@ -38,7 +38,7 @@ from synthetic import WORKLOADS, attention_inputs, bf16_bits_to_f32  # noqa: E40
 
 WORKLOAD = "long128"
 CAUSAL = True
-PASSES = ("fwd",)
+PASSES = ("fwd", "bwd")
 METRIC = "attention fwd/bwd TFLOP/s and % of B200 dense BF16/FP8 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -206,21 +206,35 @@ def run_ours(args, rank, world, local_rank):
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
+    dq = torch.empty_like(dev["q"])
+    dk = torch.empty_like(dev["k"])
+    dv = torch.empty_like(dev["v"])
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, Hq, Hkv, N, d), dtype=torch.uint8, device="cuda")
+
     def fwd():
         fa.fa_fwd(dev["q"], dev["k"], dev["v"], causal=causal, out=o, lse=lse)
+
+    def bwd():
+        fa.fa_bwd(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], causal=causal, dq=dq, dk=dk, dv=dv,
+                  workspace=ws)
+
+    def step():
+        fwd()
+        if "bwd" in passes:
+            bwd()
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     for _ in range(args.warmup):
-        fwd()
+        step()
     torch.cuda.synchronize()
     assert fa.fa_last_device_status() == 0
 
     # --- device-timed region: K steps; events around each pass on the
     # launching stream give the per-launch duration of each kernel
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
@@ -232,11 +246,15 @@ def run_ours(args, rank, world, local_rank):
             ev[i][0].record(stream)
             fwd()
             ev[i][1].record(stream)
+            if "bwd" in passes:
+                bwd()
+            ev[i][2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
     barrier()
     ms = t_start.elapsed_time(t_end)
-    fwd_ms = [a.elapsed_time(b) for a, b in ev]
+    fwd_ms = [a.elapsed_time(b_) for a, b_, _ in ev]
+    bwd_ms = [b_.elapsed_time(c) for _, b_, c in ev]
     clocks = clk.summary()
     if world > 1:
         t = torch.tensor([ms], device="cuda")
@@ -252,18 +270,22 @@ def run_ours(args, rank, world, local_rank):
         e2e_steps = min(args.steps, 50)
         o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        h2d = sum(host[n].numel() * 2 for n in ("q", "k", "v"))
-        d2h = o_host.numel() * 2 + lse_host.numel() * 4
+        ins = [n for n in ("q", "k", "v", "do") if n in host]
+        outs = [(o, o_host), (lse, lse_host)]
+        if "bwd" in passes:
+            outs += [(t, torch.empty(t.shape, dtype=t.dtype).pin_memory()) for t in (dq, dk, dv)]
+        h2d = sum(host[n].numel() * 2 for n in ins)
+        d2h = sum(h.numel() * h.element_size() for _, h in outs)
         barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(e2e_steps):
-            for n in ("q", "k", "v"):
+            for n in ins:
                 dev[n].copy_(host[n], non_blocking=True)
-            fwd()
-            o_host.copy_(o, non_blocking=True)
-            lse_host.copy_(lse, non_blocking=True)
+            step()
+            for t, h in outs:
+                h.copy_(t, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
@@ -279,8 +301,15 @@ def run_ours(args, rank, world, local_rank):
         return
     pk, pk_kind = peaks()
     peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    avg_fwd_ms = statistics.mean(fwd_ms)
-    achieved = w.fwd_flops(causal) / (avg_fwd_ms * 1e-3) / 1e12
+    fwd_tf = w.fwd_flops(causal) / (statistics.mean(fwd_ms) * 1e-3) / 1e12
+    bwd_tf = w.bwd_flops(causal) / (statistics.mean(bwd_ms) * 1e-3) / 1e12 if "bwd" in passes else None
+    # dominant kernel: the backward (2.5x the forward's FLOPs); its events
+    # bracket the whole fa_bwd call (preprocess + main + postprocess), so the
+    # figure is a lower bound for the main kernel alone
+    if "bwd" in passes:
+        dom, achieved = "fa_bwd: bwd_pre_kernel + bwd_bf16_kernel + bwd_post_kernel", bwd_tf
+    else:
+        dom, achieved = "fwd_bf16_kernel", fwd_tf
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         v, el, heads, threads = cpu_oracle_sample(w, causal, passes, seconds_budget=args.cpu_seconds)
@@ -293,13 +322,14 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": f"{args.workload}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} causal={causal}",
                    "passes": list(passes), "l2": "inputs larger than L2 (no flush between steps)",
                    "parallelism": f"replica x{world} (independent problems per GPU)"},
-        "fwd_tflops": achieved, "fwd_frac_of_peak": achieved / peak,
-        "roofline": {"bound": "tensor", "kernel": "fwd_bf16_kernel", "achieved": achieved, "peak": peak,
+        "fwd_tflops": fwd_tf, "fwd_frac_of_peak": fwd_tf / peak,
+        "bwd_tflops": bwd_tf, "bwd_frac_of_peak": (bwd_tf / peak) if bwd_tf else None,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                      "peak_kind": f"{pk_kind} bf16 dense, sustained (kernel timed inside a long loop)",
                      "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps * len(passes),
+        "gpu_launches": args.steps * (1 + (3 if "bwd" in passes else 0)),
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

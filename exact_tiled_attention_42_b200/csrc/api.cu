@@ -76,6 +76,23 @@ bool make_map_bf16(CUtensorMap* m, const void* ptr, int d, int N, long long oute
   return r == CUDA_SUCCESS;
 }
 
+// 3-D map over the fp32 dQ accumulator [BH, N, d]: 16 x 32 boxes, 64B swizzle
+// (the layout the backward's drain warps stage rows in).
+bool make_map_f32_acc(CUtensorMap* m, const void* ptr, int d, int N, long long outer) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(N) * d * 4};
+  cuuint32_t box[3] = {16, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
 }  // namespace
 
 extern "C" {
@@ -130,9 +147,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d) {
   if (check_shape(B, Hq, Hkv, N, d, 1.0f) != FA_OK) return 0;
-  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  const size_t rows = static_cast<size_t>(B) * Hq * N;
-  return up(rows * sizeof(float)) + up(rows * d * sizeof(float));
+  const size_t bh = static_cast<size_t>(B) * Hq;
+  const size_t npad = static_cast<size_t>((N + 127) / 128) * 128;
+  return 2 * up256(bh * npad * sizeof(float)) + up256(bh * N * d * sizeof(float));
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
@@ -146,9 +163,38 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < fa_bwd_workspace_size(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
-  (void)causal;
-  (void)stream;
-  return FA_ERR_UNSUPPORTED;  // backward kernel not built yet
+  const long long BH = static_cast<long long>(B) * Hq, BHkv = static_cast<long long>(B) * Hkv;
+  const int T = (N + 127) / 128;
+  if (T > 65535 || BHkv > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;  // grid = (B*Hkv, key tiles)
+  const size_t vec_bytes = up256(static_cast<size_t>(BH) * T * 128 * sizeof(float));
+  char* ws = static_cast<char*>(workspace);
+  fa::BwdParams p;
+  p.o = static_cast<const uint16_t*>(o);
+  p.dout = static_cast<const uint16_t*>(dout);
+  p.lse = lse;
+  p.delta = reinterpret_cast<float*>(ws);
+  p.neg_lse2 = reinterpret_cast<float*>(ws + vec_bytes);
+  p.dq_accum = reinterpret_cast<float*>(ws + 2 * vec_bytes);
+  p.dq = static_cast<uint16_t*>(dq);
+  p.status = status_ptr();
+  p.N = N;
+  p.Npad = T * 128;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.num_tiles = T;
+  p.d = d;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (!p.status) return FA_ERR_CUDA;
+  CUtensorMap tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmAcc;
+  if (!make_map_bf16(&tmQ, q, d, N, BH, 128) || !make_map_bf16(&tmK, k, d, N, BHkv, 128) ||
+      !make_map_bf16(&tmV, v, d, N, BHkv, 128) || !make_map_bf16(&tmdO, dout, d, N, BH, 128) ||
+      !make_map_bf16(&tmdK, dk, d, N, BHkv, 128) || !make_map_bf16(&tmdV, dv, d, N, BHkv, 128) ||
+      !make_map_f32_acc(&tmAcc, p.dq_accum, d, N, BH))
+    return FA_ERR_CUDA;
+  cudaError_t e = fa::launch_bwd_bf16(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmAcc, p, B, causal != 0, stream);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 size_t fa_fp8_workspace_size(int B, int Hq, int Hkv, int N, int d) {

@@ -1,0 +1,560 @@
+// Backward pass of exact softmax attention on sm_100a by recomputation.
+//
+// The pages say that the tiled algorithm trains Transformers faster
+// ("FlashAttention: Fast and Memory-Efficient Exact Attention with
+// IO-Awareness", abstract) but give no backward pass. The one here is the
+// analytic gradient of O = softmax(scale Q K^T) V, with P rebuilt tile by tile
+// from Q, K and the forward's log-sum-exp so that no N x N matrix is stored:
+//     P  = exp(scale S - LSE)            dV += P^T dO
+//     dP = dO V^T                        dS  = P * (dP - D),  D = rowsum(dO * O)
+//     dK += scale dS^T Q                 dQ += scale dS K
+// Three kernels: a preprocess (D, -LSE log2 e, zero the fp32 dQ accumulator),
+// the main kernel, and a postprocess (dQ = scale * accumulator -> bf16).
+//
+// Main kernel: one CTA per (128-key tile j, KV head). It keeps K_j and V_j in
+// shared memory and dK_j, dV_j in tensor memory, and loops over the query
+// heads that share the KV head and over the query tiles i (i >= j when
+// causal), so dK and dV are summed over the group without atomics. Per step,
+// everything is "transposed" so that keys sit on the 128 tensor-memory lanes:
+//   S^T  = K_j Q_i^T      (shared x shared -> tensor memory)
+//   dP^T = V_j dO_i^T     (shared x shared -> tensor memory)
+//   dV  += P^T dO_i       (P^T from tensor memory, bf16)
+//   dK  += dS^T Q_i       (dS^T from tensor memory, bf16)
+//   dQ_i = dS K_j         (dS from shared memory, MN-major)
+// Roles: warps 0-3 turn S^T into P^T and dP^T into dS^T (thread = key row);
+// warps 4-7 drain dQ_i out of tensor memory and add it into the fp32
+// accumulator with TMA reduce-add (thread = query row); warp 8 loads with TMA;
+// one thread of warp 9 issues every MMA. P^T and dS^T (bf16) are written over
+// the S^T columns; for d = 128 the dQ accumulator reuses the dP^T columns and
+// dS reuses the shared-memory slot of dO_i once dV has read it.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fa {
+namespace {
+
+constexpr int BT = 128;  // keys per CTA tile; queries per step
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int BWD_THREADS = 320;
+constexpr float LOG2E = 1.4426950408889634f;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int BOX_BYTES = 128 * 128;  // 64 bf16 columns x 128 rows
+  static constexpr int BOXES = D / 64;
+  static constexpr int TILE_BYTES = BOXES * BOX_BYTES;
+  static constexpr bool DS_ALIAS = (D == 128);
+  static constexpr int DS_BYTES = 128 * 128 * 2;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE_BYTES;
+  static constexpr int OFF_Q = OFF_V + TILE_BYTES;    // 2 slots
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE_BYTES;  // 2 slots
+  static constexpr int OFF_DS = OFF_DO + 2 * TILE_BYTES;
+  static constexpr int OFF_STG = OFF_DS + (DS_ALIAS ? 0 : DS_BYTES);  // 4 warps x 2 buffers x 2 KB
+  static constexpr int OFF_VEC = OFF_STG + 16384;  // 2 slots x (-LSE log2e, D) x 512 B
+  static constexpr int OFF_BAR = OFF_VEC + 2048;
+  static constexpr int NUM_BARS = 19;
+  static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
+  static constexpr uint32_t COL_S = 0;    // S^T; then P^T bf16 in [0,64) and dS^T bf16 in [64,128)
+  static constexpr uint32_t COL_DP = 128;
+  static constexpr uint32_t COL_DV = 256;
+  static constexpr uint32_t COL_DK = 256 + D;
+  static constexpr uint32_t COL_DQ = (D == 64) ? 384 : 128;
+  static constexpr bool DQ_SHARES_DP = (COL_DQ == COL_DP);
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct BwdBars {
+  uint32_t base;
+  __device__ uint32_t kv_full() const { return base; }
+  __device__ uint32_t q_full(int s) const { return base + 8u * (1 + s); }
+  __device__ uint32_t q_empty(int s) const { return base + 8u * (3 + s); }
+  __device__ uint32_t do_full(int s) const { return base + 8u * (5 + s); }
+  __device__ uint32_t do_empty(int s) const { return base + 8u * (7 + s); }
+  __device__ uint32_t s_full() const { return base + 8u * 9; }
+  __device__ uint32_t dp_full() const { return base + 8u * 10; }
+  __device__ uint32_t p_ready() const { return base + 8u * 11; }
+  __device__ uint32_t ds_ready() const { return base + 8u * 12; }
+  __device__ uint32_t dv_done() const { return base + 8u * 13; }
+  __device__ uint32_t dq_full() const { return base + 8u * 14; }
+  __device__ uint32_t dq_free() const { return base + 8u * 15; }
+  __device__ uint32_t dkdv_done() const { return base + 8u * 16; }
+  __device__ uint32_t epi() const { return base + 8u * 17; }
+  __device__ uint32_t teardown() const { return base + 8u * 18; }
+};
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > 100000000ull) break;  // 100 ms
+  }
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// ------------------------------------------------------------------ preprocess
+// D = rowsum(dO * O) and -LSE * log2(e) per query row (0 in the padding rows
+// up to Npad), and zeros in the fp32 dQ accumulator. d/8 lanes per row, each
+// covering 8 consecutive elements.
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p, long long total_rows) {
+  const int lpr = p.d >> 3;
+  const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long row = gt / lpr;
+  const int sub = static_cast<int>(gt - row * lpr);
+  const bool valid = row < total_rows;
+  const long long bh = valid ? row / p.Npad : 0;
+  const int n = valid ? static_cast<int>(row - bh * p.Npad) : 0;
+  const bool real = valid && n < p.N;
+  float acc = 0.f;
+  if (real) {
+    const long long off = (bh * p.N + n) * p.d + sub * 8;
+    const uint4 ov = *reinterpret_cast<const uint4*>(p.o + off);
+    const uint4 gv = *reinterpret_cast<const uint4*>(p.dout + off);
+    const uint32_t oa[4] = {ov.x, ov.y, ov.z, ov.w};
+    const uint32_t ga[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc += bf16_lo(oa[e]) * bf16_lo(ga[e]) + bf16_hi(oa[e]) * bf16_hi(ga[e]);
+    float4* z = reinterpret_cast<float4*>(p.dq_accum + off);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int off = lpr >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (valid && sub == 0) {
+    p.delta[row] = real ? acc : 0.f;
+    p.neg_lse2[row] = real ? -p.lse[bh * p.N + n] * LOG2E : 0.f;
+  }
+}
+
+// ----------------------------------------------------------------- postprocess
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq,
+                                                       long long n8, float scale) {
+  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < n8;
+       t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * t];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * t + 1];
+    uint4 o;
+    o.x = pack_bf16x2(a.x * scale, a.y * scale);
+    o.y = pack_bf16x2(a.z * scale, a.w * scale);
+    o.z = pack_bf16x2(b.x * scale, b.y * scale);
+    o.w = pack_bf16x2(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dq)[t] = o;
+  }
+}
+
+// ------------------------------------------------------------------ main kernel
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+    bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                    const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                    const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int bkv = blockIdx.x;  // b * Hkv + kvh
+  const int j = blockIdx.y;    // key tile
+  const int b = bkv / p.Hkv;
+  const int kvh = bkv - b * p.Hkv;
+  const int T = p.num_tiles;
+  const int i0 = CAUSAL ? j : 0;
+  const int nq = T - i0;
+  const int n_it = p.group * nq;
+
+  const BwdBars bars{base + C::OFF_BAR};
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_BAR + C::NUM_BARS * 8);
+  volatile int* const abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars.kv_full(), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bars.q_full(s), 1);
+      mbar_init(bars.q_empty(s), 1);
+      mbar_init(bars.do_full(s), 1);
+      mbar_init(bars.do_empty(s), 1);
+    }
+    mbar_init(bars.s_full(), 1);
+    mbar_init(bars.dp_full(), 1);
+    mbar_init(bars.p_ready(), 4);
+    mbar_init(bars.ds_ready(), 4);
+    mbar_init(bars.dv_done(), 1);
+    mbar_init(bars.dq_full(), 1);
+    mbar_init(bars.dq_free(), 4);
+    mbar_init(bars.dkdv_done(), 1);
+    mbar_init(bars.epi(), 4);
+    mbar_init(bars.teardown(), 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == PRODUCER_WARP && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmdO);
+    prefetch_tmap(&tmdQacc);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto q_head = [&](int it) { return b * p.Hq + kvh * p.group + it / nq; };  // b * Hq + hq
+  auto q_tile = [&](int it) { return i0 + it % nq; };
+  auto ds_smem = [&](int st) -> uint32_t {
+    return C::DS_ALIAS ? base + C::OFF_DO + st * C::TILE_BYTES : base + C::OFF_DS;
+  };
+
+  if (warp == PRODUCER_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bars.kv_full(), 2 * C::TILE_BYTES);
+      for (int bx = 0; bx < C::BOXES; ++bx) {
+        tma_load_3d(base + C::OFF_K + bx * C::BOX_BYTES, &tmK, bars.kv_full(), bx * 64, j * BT, bkv);
+        tma_load_3d(base + C::OFF_V + bx * C::BOX_BYTES, &tmV, bars.kv_full(), bx * 64, j * BT, bkv);
+      }
+      int issued = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        const int bhq = q_head(it);
+        const int i = q_tile(it);
+        if (!mbar_wait(bars.q_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 1)) break;
+        mbar_arrive_expect_tx(bars.q_full(st), C::TILE_BYTES + 1024);
+        for (int bx = 0; bx < C::BOXES; ++bx)
+          tma_load_3d(base + C::OFF_Q + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, bars.q_full(st), bx * 64,
+                      i * BT, bhq);
+        const long long voff = static_cast<long long>(bhq) * p.Npad + i * BT;
+        bulk_load_1d(base + C::OFF_VEC + st * 1024, p.neg_lse2 + voff, 512, bars.q_full(st));
+        bulk_load_1d(base + C::OFF_VEC + st * 1024 + 512, p.delta + voff, 512, bars.q_full(st));
+        if (!mbar_wait(bars.do_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 2)) {
+          issued = 2 * it + 1;
+          break;
+        }
+        mbar_arrive_expect_tx(bars.do_full(st), C::TILE_BYTES);
+        for (int bx = 0; bx < C::BOXES; ++bx)
+          tma_load_3d(base + C::OFF_DO + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmdO, bars.do_full(st), bx * 64,
+                      i * BT, bhq);
+        issued = 2 * it + 2;
+      }
+      if (*abort) {
+        drain_wait(bars.kv_full(), 0);
+        for (int t = (issued > 4 ? issued - 4 : 0); t < issued; ++t) {
+          const int it = t >> 1;
+          const uint32_t bar = (t & 1) ? bars.do_full(it & 1) : bars.q_full(it & 1);
+          drain_wait(bar, (it >> 1) & 1);
+        }
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      constexpr uint32_t IDESC_SS = idesc_bf16(BT, BT, false, false);
+      constexpr uint32_t IDESC_TS = idesc_bf16(BT, D, false, true);
+      constexpr uint32_t IDESC_DQ = idesc_bf16(BT, D, true, true);
+      const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
+      bool ok = mbar_wait(bars.kv_full(), 0, abort, p.status, SITE_BWD + 3);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        const uint32_t sQ = base + C::OFF_Q + st * C::TILE_BYTES;
+        const uint32_t sdO = base + C::OFF_DO + st * C::TILE_BYTES;
+        if (!mbar_wait(bars.q_full(st), ph, abort, p.status, SITE_BWD + 4)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K_j Q_i^T
+          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + C::COL_S, smem_desc_sw128(sK + off, 16, 1024), smem_desc_sw128(sQ + off, 16, 1024),
+                 IDESC_SS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bars.s_full());
+        if (!mbar_wait(bars.do_full(st), ph, abort, p.status, SITE_BWD + 5)) break;
+        if (C::DQ_SHARES_DP && it > 0 && !mbar_wait(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
+          break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V_j dO_i^T
+          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+          mma_ss(tmem + C::COL_DP, smem_desc_sw128(sV + off, 16, 1024), smem_desc_sw128(sdO + off, 16, 1024),
+                 IDESC_SS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bars.dp_full());
+        if (!mbar_wait(bars.p_ready(), it & 1, abort, p.status, SITE_BWD + 7)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BT / 16; ++kk)  // dV += P^T dO_i
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, smem_desc_sw128(sdO + kk * 2048, C::BOX_BYTES, 1024),
+                 IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bars.dv_done());
+        if (!mbar_wait(bars.ds_ready(), it & 1, abort, p.status, SITE_BWD + 8)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BT / 16; ++kk)  // dK += dS^T Q_i
+          mma_ts(tmem + C::COL_DK, tmem + C::COL_S + 64 + kk * 8, smem_desc_sw128(sQ + kk * 2048, C::BOX_BYTES, 1024),
+                 IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bars.q_empty(st));
+        if (!C::DQ_SHARES_DP && it > 0 &&
+            !mbar_wait(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
+          break;
+        tc_fence_after();
+        const uint32_t sdS = ds_smem(st);
+#pragma unroll
+        for (int kk = 0; kk < BT / 16; ++kk)  // dQ_i = dS K_j (A and B MN-major)
+          mma_ss(tmem + C::COL_DQ, smem_desc_sw128(sdS + kk * 2048, 16384, 1024),
+                 smem_desc_sw128(sK + kk * 2048, C::BOX_BYTES, 1024), IDESC_DQ, kk > 0 ? 1u : 0u);
+        mma_commit(bars.dq_full());
+        mma_commit(bars.do_empty(st));
+      }
+      mma_commit(bars.dkdv_done());
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P and dS (thread = key row)
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::COL_S;
+    const uint32_t tDP = tmem + lane_off + C::COL_DP;
+    const float cl2 = p.scale_log2;
+    bool ok = true;
+    for (int it = 0; ok && it < n_it; ++it) {
+      const int st = it & 1;
+      const uint32_t ph = (it >> 1) & 1;
+      const int i = q_tile(it);
+      ok = __all_sync(0xffffffffu, mbar_wait(bars.q_full(st), ph, abort, p.status, SITE_BWD + 9));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full(), it & 1, abort, p.status, SITE_BWD + 10));
+      if (!ok) break;
+      tc_fence_after();
+      const float* vec_lse = reinterpret_cast<const float*>(base_ptr + C::OFF_VEC + st * 1024);
+      const float* vec_d = vec_lse + 128;
+      uint32_t pk[64];
+      {
+        float s[BT];
+#pragma unroll
+        for (int c = 0; c < BT; c += 32) {
+          uint32_t t[32];
+          tmem_ld_x32(tS + c, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[c + e] = __uint_as_float(t[e]);
+        }
+#pragma unroll
+        for (int c = 0; c < BT; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(vec_lse + c);
+          s[c] = ex2(fmaf(s[c], cl2, l4.x));
+          s[c + 1] = ex2(fmaf(s[c + 1], cl2, l4.y));
+          s[c + 2] = ex2(fmaf(s[c + 2], cl2, l4.z));
+          s[c + 3] = ex2(fmaf(s[c + 3], cl2, l4.w));
+        }
+        if (CAUSAL && i == j) {  // diagonal tile: key r sees queries c >= r
+#pragma unroll
+          for (int c = 0; c < BT; ++c)
+            if (c < r) s[c] = 0.f;
+        }
+        const int qlim = p.N - i * BT;  // queries past N are padding
+        if (qlim < BT) {
+#pragma unroll
+          for (int c = 0; c < BT; ++c)
+            if (c >= qlim) s[c] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 64; ++e) pk[e] = pack_bf16x2(s[2 * e], s[2 * e + 1]);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t t[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) t[e] = pk[c * 16 + e];
+        tmem_st_x16(tS + c * 16, t);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.p_ready());
+
+      ok = __all_sync(0xffffffffu, mbar_wait(bars.dp_full(), it & 1, abort, p.status, SITE_BWD + 11));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.dv_done(), it & 1, abort, p.status, SITE_BWD + 12));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t sdS = ds_smem(st);
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t t[32];
+        tmem_ld_x32(tDP + cc * 32, t);
+        tmem_wait_ld();
+        uint32_t dsk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = cc * 32 + 2 * e;
+          const float2 dd = *reinterpret_cast<const float2*>(vec_d + c);
+          const uint32_t pp = pk[cc * 16 + e];
+          dsk[e] = pack_bf16x2(bf16_lo(pp) * (__uint_as_float(t[2 * e]) - dd.x),
+                               bf16_hi(pp) * (__uint_as_float(t[2 * e + 1]) - dd.y));
+        }
+        tmem_st_x16(tS + 64 + cc * 16, dsk);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t addr = sdS + (cc >> 1) * C::BOX_BYTES + sw128_offset(r, (cc & 1) * 4 + q);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dsk[4 * q]), "r"(dsk[4 * q + 1]),
+                       "r"(dsk[4 * q + 2]), "r"(dsk[4 * q + 3])
+                       : "memory");
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.ds_ready());
+    }
+    // ------------------------------------------------------------ dK, dV epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.dkdv_done(), 0, abort, p.status, SITE_BWD + 13));
+    if (ok) {
+      tc_fence_after();
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t src = tmem + lane_off + (which ? C::COL_DV : C::COL_DK);
+        const float mul = which ? 1.0f : p.scale;
+        const uint32_t stage = base + C::OFF_Q + which * C::TILE_BYTES;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t t[32];
+          tmem_ld_x32(src + c, t);
+          tmem_wait_ld();
+          const uint32_t box = stage + (c >> 6) * C::BOX_BYTES;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w4[e] = pack_bf16x2(__uint_as_float(t[q * 8 + 2 * e]) * mul, __uint_as_float(t[q * 8 + 2 * e + 1]) * mul);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(box + sw128_offset(r, ((c & 63) >> 3) + q)),
+                         "r"(w4[0]), "r"(w4[1]), "r"(w4[2]), "r"(w4[3])
+                         : "memory");
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.epi());
+      if (r == 0 && mbar_wait(bars.epi(), 0, abort, p.status, SITE_BWD + 14)) {
+        for (int bx = 0; bx < C::BOXES; ++bx) {
+          tma_store_3d(&tmdK, base + C::OFF_Q + bx * C::BOX_BYTES, bx * 64, j * BT, bkv);
+          tma_store_3d(&tmdV, base + C::OFF_Q + C::TILE_BYTES + bx * C::BOX_BYTES, bx * 64, j * BT, bkv);
+        }
+        bulk_commit();
+        bulk_wait_read0();
+      }
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ dQ drain (thread = query row)
+    const int w = warp & 3;
+    const uint32_t tDQ = tmem + (static_cast<uint32_t>(w * 32) << 16) + C::COL_DQ;
+    const uint32_t stg0 = base + C::OFF_STG + w * 2 * 2048;
+    int cnt = 0;
+    bool ok = true;
+    for (int it = 0; ok && it < n_it; ++it) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bars.dq_full(), it & 1, abort, p.status, SITE_BWD + 15));
+      if (!ok) break;
+      tc_fence_after();
+      float acc[D];
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t t[32];
+        tmem_ld_x32(tDQ + c, t);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[c + e] = __uint_as_float(t[e]);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.dq_free());
+      const int bhq = q_head(it);
+      const int row0 = q_tile(it) * BT + w * 32;
+      if (row0 >= p.N) continue;  // every row of this warp is padding
+#pragma unroll
+      for (int c16 = 0; c16 < D / 16; ++c16) {
+        const uint32_t buf = stg0 + (cnt & 1) * 2048;
+        if (lane == 0) bulk_wait_read<1>();  // the reduce that last read this buffer is done with it
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t addr = buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4);
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(acc[c16 * 16 + 4 * q]),
+                       "f"(acc[c16 * 16 + 4 * q + 1]), "f"(acc[c16 * 16 + 4 * q + 2]), "f"(acc[c16 * 16 + 4 * q + 3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tmdQacc, buf, c16 * 16, row0, bhq);
+          bulk_commit();
+        }
+        ++cnt;
+      }
+    }
+    if (lane == 0) bulk_wait0();
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    if (*abort) {
+      if (lane == 0) {
+        mma_commit(bars.teardown());
+        drain_wait(bars.teardown(), 0);
+      }
+      __syncwarp();
+    }
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_main(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                        const CUtensorMap& tmdO, const CUtensorMap& tmdK, const CUtensorMap& tmdV,
+                        const CUtensorMap& tmdQacc, const BwdParams& p, int B, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  auto kern = bwd_bf16_kernel<D, CAUSAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  dim3 grid(B * p.Hkv, p.num_tiles);  // key tile j = blockIdx.y: longest causal loops launch first
+  kern<<<grid, BWD_THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_bf16(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                            const CUtensorMap& tmdO, const CUtensorMap& tmdK, const CUtensorMap& tmdV,
+                            const CUtensorMap& tmdQacc, const BwdParams& p, int B, bool causal,
+                            cudaStream_t stream) {
+  const long long BH = static_cast<long long>(B) * p.Hq;
+  const long long rows = BH * p.Npad;
+  const long long threads = rows * (p.d / 8);
+  bwd_pre_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p, rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (p.d == 64)
+    e = causal ? launch_main<64, true>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream)
+               : launch_main<64, false>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream);
+  else
+    e = causal ? launch_main<128, true>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream)
+               : launch_main<128, false>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream);
+  if (e != cudaSuccess) return e;
+  const long long n8 = BH * p.N * p.d / 8;
+  long long blocks = (n8 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  bwd_post_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p.dq_accum, p.dq, n8, p.scale);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cstdint>
 
 namespace fa {
 
@@ -22,6 +23,35 @@ struct FwdParams {
 // 64-column x 128-row boxes and 128-byte swizzle.
 cudaError_t launch_fwd_bf16(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const CUtensorMap& tmO, const FwdParams& p, int BH, int d, bool causal,
+                            cudaStream_t stream);
+
+struct BwdParams {
+  const uint16_t* o;     // bf16 [B*Hq, N, d]   (preprocess)
+  const uint16_t* dout;  // bf16 [B*Hq, N, d]   (preprocess)
+  const float* lse;      // [B*Hq, N], natural log (preprocess)
+  float* delta;          // workspace [B*Hq, Npad]: D = rowsum(dO * O), 0 past N
+  float* neg_lse2;       // workspace [B*Hq, Npad]: -LSE * log2(e), 0 past N
+  float* dq_accum;       // workspace [B*Hq, N, d] fp32, zeroed by the preprocess
+  uint16_t* dq;          // bf16 [B*Hq, N, d]   (postprocess)
+  int* status;
+  int N;
+  int Npad;              // num_qtiles * 128
+  int Hq;
+  int Hkv;
+  int group;
+  int num_tiles;         // ceil(N / 128): query tiles and key tiles
+  int d;
+  float scale;
+  float scale_log2;
+};
+
+// Backward: preprocess (D, -LSE*log2 e, zero dq_accum), the main kernel over
+// (key tile, KV head), and the dq postprocess. tmQ/tmdO: [B*Hq, N, d] bf16;
+// tmK/tmV/tmdK/tmdV: [B*Hkv, N, d] bf16 (64 x 128 boxes, 128B swizzle);
+// tmdQacc: fp32 [B*Hq, N, d] with 16 x 32 boxes and 64B swizzle.
+cudaError_t launch_bwd_bf16(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                            const CUtensorMap& tmdO, const CUtensorMap& tmdK, const CUtensorMap& tmdV,
+                            const CUtensorMap& tmdQacc, const BwdParams& p, int B, bool causal,
                             cudaStream_t stream);
 
 }  // namespace fa
