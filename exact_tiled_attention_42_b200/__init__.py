@@ -11,6 +11,7 @@ from .api import (  # noqa: F401
     FA_OK,
     fa_fwd,
     fa_bwd,
+    fa_bwd_noalloc,
     fa_fwd_fp8,
     fa_bwd_workspace_size,
     fa_fp8_workspace_size,

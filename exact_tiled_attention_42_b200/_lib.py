@@ -22,6 +22,7 @@ SIGNATURES = {
     "fa_fwd": (_c_int, [_c_void_p] * 5 + [_c_int] * 6 + [_c_float, _c_void_p]),
     "fa_bwd_workspace_size": (_c_size_t, [_c_int] * 5),
     "fa_bwd": (_c_int, [_c_void_p] * 10 + [_c_size_t] + [_c_int] * 6 + [_c_float, _c_void_p]),
+    "fa_bwd_noalloc": (_c_int, [_c_void_p] * 9 + [_c_int] * 6 + [_c_float, _c_void_p]),
     "fa_fp8_workspace_size": (_c_size_t, [_c_int] * 5),
     "fa_fwd_fp8": (_c_int, [_c_void_p] * 5 + [_c_uint64, _c_int, _c_void_p, _c_size_t] + [_c_int] * 6
                    + [_c_float, _c_void_p]),

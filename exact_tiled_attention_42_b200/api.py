@@ -113,6 +113,31 @@ def fa_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = No
     return dq, dk, dv
 
 
+def fa_bwd_noalloc(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+                   dq=None, dk=None, dv=None, stream=None):
+    """fa_bwd without a workspace argument: the library's built-in scratch
+    (at most FA_BWD_NOALLOC_MAX_BYTES) is used instead. For callers that
+    cannot allocate device memory at the call; calls that may run
+    concurrently on the GPU must be serialised because they share the
+    scratch."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    for name, t, shp in (("q", q, (B, Hq, N, d)), ("k", k, (B, Hkv, N, d)), ("v", v, (B, Hkv, N, d)),
+                         ("o", o, (B, Hq, N, d)), ("dout", dout, (B, Hq, N, d))):
+        _check(name, t, torch.bfloat16, shp)
+    _check("lse", lse, torch.float32, (B, Hq, N))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = _lib.load().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                    dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                    B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    if st != FA_OK:
+        raise FAError("fa_bwd_noalloc", st)
+    return dq, dk, dv
+
+
 def fa_fwd_fp8(q, k, v, causal: bool = False, scale: float | None = None, rotation_seed: int = 0,
                use_rotation: bool = True, out=None, lse=None, workspace=None, stream=None):
     """FP8 (e4m3) forward with 64-row block scales and optional Hadamard

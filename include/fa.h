@@ -28,7 +28,9 @@
  *   - Calls are asynchronous on `stream` (0 = legacy default stream), like a
  *     kernel launch; outputs are valid once the stream has been synchronised.
  *   - The caller owns every buffer, workspaces included. The library allocates
- *     no device memory and keeps no state between calls.
+ *     no device memory and keeps no state between calls (fa_bwd_noalloc's
+ *     built-in scratch array, described at its declaration, is the one
+ *     exception).
  *   - Every argument is checked before anything is launched; a failed check
  *     returns an error and launches nothing. A launch error is returned as
  *     FA_ERR_CUDA.
@@ -83,6 +85,37 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* workspace, size_t workspace_bytes,
                  int B, int Hq, int Hkv, int N, int d, int causal, float scale,
                  cudaStream_t stream);
+
+/*
+ * Largest scratch, in bytes, that fa_bwd_noalloc can use (32 MiB). It is
+ * enough for B*Hq*N up to about 63,000 query rows at d = 128 (126,000 at d = 64).
+ */
+#define FA_BWD_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
+
+/*
+ * Backward pass that needs no workspace from the caller. The pages have no
+ * counterpart: this is a convenience of the library, not part of the method.
+ * It is fa_bwd with its scratch (D, -LSE log2 e and the fp32 dQ accumulator)
+ * taken from a fixed array of FA_BWD_NOALLOC_MAX_BYTES inside the library's
+ * device memory, held on every GPU that loads the library until the process
+ * exits. It is meant for callers that cannot allocate device memory at the
+ * point of the call (C code with no device allocator of its own, or code
+ * that must not call cudaMalloc/cudaFree there because they synchronise the
+ * device). Arguments, layouts and results are those of fa_bwd.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree.
+ *   - Returns FA_ERR_WORKSPACE, launching nothing, when fa_bwd_workspace_size
+ *     for these sizes exceeds FA_BWD_NOALLOC_MAX_BYTES.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the one array. Each call rewrites every scratch value it
+ *     reads, so leftovers from earlier calls do not matter, but calls that can
+ *     run at the same time on the GPU (other streams, other threads) race and
+ *     must be serialised by the caller.
+ */
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv,
+                         int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                         cudaStream_t stream);
 
 /*
  * Bytes of device workspace fa_fwd_fp8 needs: e4m3 copies of Q, K, V
