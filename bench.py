@@ -297,6 +297,9 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
     assert fa.fa_last_device_status() == 0
 
+    fp8 = None if args.no_fp8 else run_fp8_leg(args, fa, stream)
+    assert fa.fa_last_device_status() == 0
+
     if rank != 0:
         return
     pk, pk_kind = peaks()
@@ -329,10 +332,49 @@ def run_ours(args, rank, world, local_rank):
                      "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None},
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "fp8": fp8,
         "gpu_launches": args.steps * (1 + (3 if "bwd" in passes else 0)),
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
+
+
+def run_fp8_leg(args, fa, stream):
+    """The FP8 forward on its own workload (B=1, H=16, N=16384, d=128,
+    non-causal, 0.1% entry outliers), timed with events around each
+    fa_fwd_fp8 call (quantisation pre-pass + FP8 forward)."""
+    import torch
+    w = WORKLOADS["fp8"]
+    causal = w.causal[0]
+    bits = attention_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, outlier_rate=w.outlier_rate, with_dout=False)
+    dev = {n: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda() for n, a in bits.items()}
+    o = torch.empty_like(dev["q"])
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device="cuda")
+    ws = torch.empty(fa.fa_fp8_workspace_size(w.B, w.Hq, w.Hkv, w.N, w.d), dtype=torch.uint8, device="cuda")
+
+    def call():
+        fa.fa_fwd_fp8(dev["q"], dev["k"], dev["v"], causal=causal, rotation_seed=w.seed, use_rotation=True,
+                      out=o, lse=lse, workspace=ws)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 300))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b_ in ev:
+        a.record(stream)
+        call()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b_) for a, b_ in ev)
+    pk, pk_kind = peaks()
+    fp8_peak = 2.0 * pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    tf = w.fwd_flops(causal) / (ms * 1e-3) / 1e12
+    return {"workload": f"fp8: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} causal={causal} e4m3",
+            "tflops": tf, "ms_per_call": ms, "calls": steps,
+            "peak": fp8_peak, "peak_kind": f"{pk_kind} bf16 dense sustained x 2 (nominal fp8:bf16 ratio)",
+            "frac_of_peak": tf / fp8_peak,
+            "includes": "quantisation pre-pass (Hadamard rotation, 64-row block scales) + FP8 forward"}
 
 
 def main():
@@ -344,6 +386,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward leg")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS),
                     help="workload to run (profiling of other shapes; the headline is the default)")
     args = ap.parse_args()

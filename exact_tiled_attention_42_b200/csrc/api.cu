@@ -92,6 +92,21 @@ bool make_map_f32_acc(CUtensorMap* m, const void* ptr, int d, int N, long long o
 }
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+size_t up1024(size_t x) { return (x + 1023) & ~static_cast<size_t>(1023); }
+
+// 3-D map over an e4m3 [outer, N, d] tensor: 128 x 128 boxes, 128B swizzle.
+bool make_map_e4m3(CUtensorMap* m, const void* ptr, int d, int N, long long outer) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N) * d};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 }  // namespace
 
@@ -199,10 +214,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
 
 size_t fa_fp8_workspace_size(int B, int Hq, int Hkv, int N, int d) {
   if (check_shape(B, Hq, Hkv, N, d, 1.0f) != FA_OK) return 0;
-  auto up = [](size_t x) { return (x + 1023) & ~static_cast<size_t>(1023); };
   const size_t nb = (N + 63) / 64;
   const size_t q = static_cast<size_t>(B) * Hq, kv = static_cast<size_t>(B) * Hkv;
-  return up(q * N * d) + 2 * up(kv * N * d) + up(q * nb * 4) + 2 * up(kv * nb * 4);
+  return up1024(q * N * d) + 2 * up1024(kv * N * d) + up1024(q * nb * 4) + 2 * up1024(kv * nb * 4);
 }
 
 fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, uint64_t rotation_seed,
@@ -211,13 +225,49 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   fa_status st = check_shape(B, Hq, Hkv, N, d, scale);
   if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;  // the FP8 kernels are built for d = 128
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < fa_fp8_workspace_size(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
-  (void)rotation_seed;
-  (void)use_rotation;
-  (void)causal;
-  (void)stream;
-  return FA_ERR_UNSUPPORTED;  // FP8 kernels not built yet
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  const long long BH = static_cast<long long>(B) * Hq, BHkv = static_cast<long long>(B) * Hkv;
+  const int nb = (N + 63) / 64;
+  if (BH > 65535) return FA_ERR_UNSUPPORTED;  // pre-pass grid.y
+  char* ws = static_cast<char*>(workspace);
+  const size_t cq = up1024(static_cast<size_t>(BH) * N * d), ckv = up1024(static_cast<size_t>(BHkv) * N * d);
+  const size_t sq = up1024(static_cast<size_t>(BH) * nb * 4), skv = up1024(static_cast<size_t>(BHkv) * nb * 4);
+  fa::Fp8Params p;
+  p.src[0] = static_cast<const uint16_t*>(q);
+  p.src[1] = static_cast<const uint16_t*>(k);
+  p.src[2] = static_cast<const uint16_t*>(v);
+  p.codes[0] = reinterpret_cast<uint8_t*>(ws);
+  p.codes[1] = reinterpret_cast<uint8_t*>(ws + cq);
+  p.codes[2] = reinterpret_cast<uint8_t*>(ws + cq + ckv);
+  p.scales[0] = reinterpret_cast<float*>(ws + cq + 2 * ckv);
+  p.scales[1] = reinterpret_cast<float*>(ws + cq + 2 * ckv + sq);
+  p.scales[2] = reinterpret_cast<float*>(ws + cq + 2 * ckv + sq + skv);
+  p.heads[0] = static_cast<int>(BH);
+  p.heads[1] = static_cast<int>(BHkv);
+  p.heads[2] = static_cast<int>(BHkv);
+  p.rotation_seed = rotation_seed;
+  p.rotate = use_rotation != 0;
+  p.lse = lse;
+  p.status = status_ptr();
+  p.N = N;
+  p.nblk = nb;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.num_qtiles = (N + 127) / 128;
+  p.num_pairs = (p.num_qtiles + 1) / 2;
+  p.score_log2 = scale * 1.4426950408889634f / (p.rotate ? static_cast<float>(d) : 1.0f);
+  if (!p.status) return FA_ERR_CUDA;
+  CUtensorMap tmQ, tmK, tmV, tmO;
+  if (!make_map_e4m3(&tmQ, p.codes[0], d, N, BH) || !make_map_e4m3(&tmK, p.codes[1], d, N, BHkv) ||
+      !make_map_e4m3(&tmV, p.codes[2], d, N, BHkv) || !make_map_bf16(&tmO, o, d, N, BH, 128))
+    return FA_ERR_CUDA;
+  cudaError_t e = fa::launch_fp8_quant(p, stream);
+  if (e == cudaSuccess) e = fa::launch_fwd_fp8(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), causal != 0, stream);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -1,0 +1,403 @@
+// FP8 (e4m3) forward of exact softmax attention on sm_100a, d = 128.
+//
+// Same CTA layout as the bf16 forward (two 128-row query tiles, TMA producer
+// warp, one MMA-issuing thread, two softmax warpgroups), on the operands the
+// FP8 pre-pass wrote: e4m3 Q and K (rotated) and V, each with one fp32 scale
+// per 64-row block. "FlashAttention-3: Fast and Accurate Attention with
+// Asynchrony and Low-precision" (abstract) describes FP8 with block
+// quantisation; the forms used here:
+//   S = sQ(row block) sK(key block) (Qc Kc^T) scale / d       (kind::f8f6f4)
+//   running max and sum as in the bf16 path, but the max is raised on every
+//   increase so P <= 1;
+//   P~ = e4m3(P * sV(key block) / max sV * 256)               (V's block scale
+//        folded into P so that one MMA sums over key blocks with different
+//        scales; the 256 keeps small probabilities above e4m3's subnormals)
+//   O = (sum P~ Vc) * max sV / 256 / l,   l = sum of unquantised P.
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512); P~ (4 e4m3 per
+// column) over the first 32 columns of its S.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fa {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int D = 128;
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int THREADS = 320;
+constexpr float LN2 = 0.69314718055994530942f;
+constexpr float P_LIFT = 256.f;
+
+struct Cfg {
+  static constexpr int TILE_BYTES = BM * D;  // e4m3: 128 rows x 128 bytes
+  static constexpr int NS = 3;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = 2 * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
+  static constexpr int OFF_O = OFF_V + NS * TILE_BYTES;  // bf16 output staging, 2 x 32 KB
+  static constexpr int O_TILE_BYTES = BM * D * 2;
+  static constexpr int OFF_BAR = OFF_O + 2 * O_TILE_BYTES;
+  static constexpr int NUM_BARS = 1 + 4 * NS + 9;
+  static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 384;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct Bars {
+  uint32_t base;
+  __device__ uint32_t q_full() const { return base; }
+  __device__ uint32_t k_full(int s) const { return base + 8u * (1 + s); }
+  __device__ uint32_t k_empty(int s) const { return base + 8u * (1 + Cfg::NS + s); }
+  __device__ uint32_t v_full(int s) const { return base + 8u * (1 + 2 * Cfg::NS + s); }
+  __device__ uint32_t v_empty(int s) const { return base + 8u * (1 + 3 * Cfg::NS + s); }
+  __device__ uint32_t s_full(int x) const { return base + 8u * (1 + 4 * Cfg::NS + x); }
+  __device__ uint32_t p_full(int x) const { return base + 8u * (3 + 4 * Cfg::NS + x); }
+  __device__ uint32_t o_done(int x) const { return base + 8u * (5 + 4 * Cfg::NS + x); }
+  __device__ uint32_t teardown() const { return base + 8u * (7 + 4 * Cfg::NS); }
+  __device__ uint32_t epi(int x) const { return base + 8u * (8 + 4 * Cfg::NS + x); }
+};
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > 100000000ull) break;  // 100 ms
+  }
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  uint16_t lo, hi;
+  asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tmov.b16 %0, t;\n\t}" : "=h"(lo) : "f"(b), "f"(a));
+  asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tmov.b16 %0, t;\n\t}" : "=h"(hi) : "f"(d), "f"(c));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <bool CAUSAL>
+__global__ void __launch_bounds__(THREADS, 1)
+    fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const Fp8Params p) {
+  using C = Cfg;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int bh = blockIdx.x;
+  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.y);
+  const int b = bh / p.Hq;
+  const int hq = bh - b * p.Hq;
+  const int kvh = b * p.Hkv + hq / p.group;
+  const int qt0 = 2 * pair, qt1 = 2 * pair + 1;
+  const bool has1 = qt1 < p.num_qtiles;
+  const int n0 = CAUSAL ? qt0 + 1 : p.num_qtiles;
+  const int n1 = has1 ? (CAUSAL ? qt1 + 1 : p.num_qtiles) : 0;
+  const int nkv = n0 > n1 ? n0 : n1;
+
+  const Bars bars{base + C::OFF_BAR};
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_BAR + C::NUM_BARS * 8);
+  volatile int* const abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars.q_full(), 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bars.k_full(s), 1);
+      mbar_init(bars.k_empty(s), 1);
+      mbar_init(bars.v_full(s), 1);
+      mbar_init(bars.v_empty(s), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bars.s_full(x), 1);
+      mbar_init(bars.p_full(x), 4);
+      mbar_init(bars.o_done(x), 1);
+      mbar_init(bars.epi(x), 4);
+    }
+    mbar_init(bars.teardown(), 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == PRODUCER_WARP && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == PRODUCER_WARP) {
+    if (lane == 0) {
+      const uint32_t sQ = base + C::OFF_Q;
+      mbar_arrive_expect_tx(bars.q_full(), (has1 ? 2 : 1) * C::TILE_BYTES);
+      tma_load_3d(sQ, &tmQ, bars.q_full(), 0, qt0 * BM, bh);
+      if (has1) tma_load_3d(sQ + C::TILE_BYTES, &tmQ, bars.q_full(), 0, qt1 * BM, bh);
+      int issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % C::NS;
+        const uint32_t ph = (j / C::NS) & 1;
+        if (!mbar_wait(bars.k_empty(s), ph ^ 1, abort, p.status, SITE_K_EMPTY)) break;
+        mbar_arrive_expect_tx(bars.k_full(s), C::TILE_BYTES);
+        tma_load_3d(base + C::OFF_K + s * C::TILE_BYTES, &tmK, bars.k_full(s), 0, j * BN, kvh);
+        if (!mbar_wait(bars.v_empty(s), ph ^ 1, abort, p.status, SITE_V_EMPTY)) {
+          issued = 2 * j + 1;
+          break;
+        }
+        mbar_arrive_expect_tx(bars.v_full(s), C::TILE_BYTES);
+        tma_load_3d(base + C::OFF_V + s * C::TILE_BYTES, &tmV, bars.v_full(s), 0, j * BN, kvh);
+        issued = 2 * j + 2;
+      }
+      if (*abort) {
+        drain_wait(bars.q_full(), 0);
+        for (int t = (issued > 2 * C::NS ? issued - 2 * C::NS : 0); t < issued; ++t) {
+          const int j = t >> 1;
+          drain_wait((t & 1) ? bars.v_full(j % C::NS) : bars.k_full(j % C::NS), (j / C::NS) & 1);
+        }
+      }
+    }
+  } else if (warp == MMA_WARP) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_QK = idesc_e4m3(BM, BN, false, false);
+      constexpr uint32_t IDESC_PV = idesc_e4m3(BM, D, false, true);
+      const uint32_t sQ = base + C::OFF_Q;
+      auto issue_qk = [&](int x, int stage) {
+        const uint32_t dS = tmem + (x ? C::COL_S1 : C::COL_S0);
+        const uint32_t qa = sQ + x * C::TILE_BYTES;
+        const uint32_t kb = base + C::OFF_K + stage * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk)  // 32 e4m3 = 32 bytes of each 128-byte row
+          mma_ss_f8(dS, smem_desc_sw128(qa + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 32, 16, 1024), IDESC_QK,
+                    kk > 0 ? 1u : 0u);
+      };
+      auto issue_pv = [&](int x, int stage, bool accumulate) {
+        const uint32_t dO = tmem + (x ? C::COL_O1 : C::COL_O0);
+        const uint32_t aP = tmem + (x ? C::COL_S1 : C::COL_S0);
+        const uint32_t vb = base + C::OFF_V + stage * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 32; ++kk)  // 32 keys = four 8-row groups; 32 e4m3 of P = 8 columns
+          mma_ts_f8(dO, aP + kk * 8, smem_desc_sw128(vb + kk * 4096, 16384, 1024), IDESC_PV,
+                    (accumulate || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&
+                mbar_wait(bars.k_full(0), 0, abort, p.status, SITE_K_FULL);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        mma_commit(bars.s_full(0));
+        if (n1 > 0) {
+          issue_qk(1, 0);
+          mma_commit(bars.s_full(1));
+        }
+        mma_commit(bars.k_empty(0));
+      }
+      for (int j = 1; ok && j <= nkv; ++j) {
+        const int vs = (j - 1) % C::NS;
+        const int ks = j % C::NS;
+        if (!mbar_wait(bars.v_full(vs), ((j - 1) / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
+        if (j < nkv && !mbar_wait(bars.k_full(ks), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) break;
+        tc_fence_after();
+        for (int x = 0; x < 2; ++x) {
+          const int nx = x ? n1 : n0;
+          if (j - 1 >= nx) continue;
+          if (!mbar_wait(bars.p_full(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(x, vs, j > 1);
+          if (j < nx) {
+            issue_qk(x, ks);
+            mma_commit(bars.s_full(x));
+          } else {
+            mma_commit(bars.o_done(x));
+          }
+        }
+        if (!ok) break;
+        if (j < nkv) mma_commit(bars.k_empty(ks));
+        mma_commit(bars.v_empty(vs));
+      }
+    }
+  } else if (warp < 8) {
+    const int x = warp >> 2;
+    const int qt = x ? qt1 : qt0;
+    const int n = x ? n1 : n0;
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int qrow = qt * BM + row;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (x ? C::COL_S1 : C::COL_S0);
+    const uint32_t tO = tmem + lane_off + (x ? C::COL_O1 : C::COL_O0);
+    const float* sQs = p.scales[0] + static_cast<long long>(bh) * p.nblk;
+    const float* sKs = p.scales[1] + static_cast<long long>(kvh) * p.nblk;
+    const float* sVs = p.scales[2] + static_cast<long long>(kvh) * p.nblk;
+    // the head's largest V block scale (every lane computes it; L1-served)
+    float vmax = 0.f;
+    for (int i = lane; i < p.nblk; i += 32) vmax = fmaxf(vmax, sVs[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+    const float wlift = P_LIFT / vmax;
+    const float crow = p.score_log2 * sQs[min(qrow, p.N - 1) >> 6];
+    float m = -INFINITY;
+    float l = 0.f;
+    bool ok = n > 0;
+    for (int j = 0; ok && j < n; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bars.s_full(x), j & 1, abort, p.status, SITE_S_FULL))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[BN];
+#pragma unroll
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld_x32(tS + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(r[i]);
+      }
+      const int kb0 = 2 * j;  // key blocks of this tile: 2j (keys 0-63) and 2j+1 (64-127)
+      const int kb1 = min(2 * j + 1, p.nblk - 1);
+      const float f0 = crow * sKs[kb0], f1 = crow * sKs[kb1];
+      const float w0 = sVs[kb0] * wlift, w1 = sVs[kb1] * wlift;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) s[c] *= (c < 64 ? f0 : f1);
+      const int kv0 = j * BN;
+      const bool edge = (kv0 + BN > p.N) || (CAUSAL && kv0 + BN - 1 > qt * BM);
+      if (edge) {
+        const int lim = CAUSAL ? min(qrow + 1, p.N) : p.N;
+#pragma unroll
+        for (int c = 0; c < BN; ++c)
+          if (kv0 + c >= lim) s[c] = -INFINITY;
+      }
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+      const float tile_max = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      if (j == 0) {
+        m = tile_max;
+      } else if (__any_sync(0xffffffffu, tile_max > m)) {
+        const float m_new = fmaxf(m, tile_max);
+        const float alpha = ex2(m - m_new);
+        l *= alpha;
+        m = m_new;
+#pragma unroll
+        for (int c = 0; c < D; c += 16) {
+          uint32_t r[16];
+          tmem_ld_x16(tO + c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st_x16(tO + c, r);
+        }
+      }
+      const float neg_m = (m == -INFINITY) ? 0.f : -m;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float w = i < 16 ? w0 : w1;
+        const float a0 = ex2(s[4 * i] + neg_m), a1 = ex2(s[4 * i + 1] + neg_m);
+        const float a2 = ex2(s[4 * i + 2] + neg_m), a3 = ex2(s[4 * i + 3] + neg_m);
+        ls[i & 3] += (a0 + a1) + (a2 + a3);
+        pk[i] = e4m3x4(a0 * w, a1 * w, a2 * w, a3 * w);
+      }
+      tmem_st_x32(tS, pk);
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.p_full(x));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.o_done(x), 0, abort, p.status, SITE_O_DONE));
+    if (ok) {
+      tc_fence_after();
+      const float out_mul = vmax / P_LIFT / l;
+      const uint32_t stage = base + C::OFF_O + x * C::O_TILE_BYTES;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        tmem_ld_x32(tO + c, r);
+        tmem_wait_ld();
+        const uint32_t box = stage + (c >> 6) * (BM * 128);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w4[e] = pack_bf16x2(__uint_as_float(r[q * 8 + 2 * e]) * out_mul,
+                                __uint_as_float(r[q * 8 + 2 * e + 1]) * out_mul);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(box + sw128_offset(row, ((c & 63) >> 3) + q)),
+                       "r"(w4[0]), "r"(w4[1]), "r"(w4[2]), "r"(w4[3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.epi(x));
+      if (row == 0 && mbar_wait(bars.epi(x), 0, abort, p.status, SITE_O_DONE)) {
+        tma_store_3d(&tmO, stage, 0, qt * BM, bh);
+        tma_store_3d(&tmO, stage + BM * 128, 64, qt * BM, bh);
+        bulk_commit();
+        bulk_wait_read0();
+      }
+      if (qrow < p.N) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(l)) * LN2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    if (*abort) {
+      if (lane == 0) {
+        mma_commit(bars.teardown());
+        drain_wait(bars.teardown(), 0);
+      }
+      __syncwarp();
+    }
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <bool CAUSAL>
+cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
+                   const Fp8Params& p, int BH, cudaStream_t stream) {
+  auto kern = fwd_fp8_kernel<CAUSAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  dim3 grid(BH, p.num_pairs);
+  kern<<<grid, THREADS, Cfg::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmO, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_fp8(const CUtensorMap& tmQ8, const CUtensorMap& tmK8, const CUtensorMap& tmV8,
+                           const CUtensorMap& tmO, const Fp8Params& p, int BH, bool causal, cudaStream_t stream) {
+  return causal ? launch<true>(tmQ8, tmK8, tmV8, tmO, p, BH, stream)
+                : launch<false>(tmQ8, tmK8, tmV8, tmO, p, BH, stream);
+}
+
+}  // namespace fa

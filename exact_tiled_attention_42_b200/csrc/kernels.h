@@ -54,4 +54,32 @@ cudaError_t launch_bwd_bf16(const CUtensorMap& tmQ, const CUtensorMap& tmK, cons
                             const CUtensorMap& tmdQacc, const BwdParams& p, int B, bool causal,
                             cudaStream_t stream);
 
+struct Fp8Params {
+  // pre-pass
+  const uint16_t* src[3];  // bf16 Q [B*Hq, N, d], K and V [B*Hkv, N, d]
+  uint8_t* codes[3];       // e4m3 copies (Q and K rotated when rotate != 0)
+  float* scales[3];        // one fp32 scale per 64-row block: [B*H, nblk]
+  int heads[3];            // B*Hq, B*Hkv, B*Hkv
+  uint64_t rotation_seed;
+  int rotate;
+  // forward
+  float* lse;              // [B*Hq, N]
+  int* status;
+  int N;
+  int nblk;                // ceil(N / 64)
+  int Hq;
+  int Hkv;
+  int group;
+  int num_qtiles;
+  int num_pairs;
+  float score_log2;        // scale * log2(e), divided by d when rotated
+};
+
+// Pre-pass (rotation + block quantisation of Q, K, V) then the FP8 forward.
+// tmQ8/tmK8/tmV8: e4m3 [B*H, N, d] with 128 x 128 boxes and 128B swizzle;
+// tmO: bf16 output map as for the bf16 forward.
+cudaError_t launch_fp8_quant(const Fp8Params& p, cudaStream_t stream);
+cudaError_t launch_fwd_fp8(const CUtensorMap& tmQ8, const CUtensorMap& tmK8, const CUtensorMap& tmV8,
+                           const CUtensorMap& tmO, const Fp8Params& p, int BH, bool causal, cudaStream_t stream);
+
 }  // namespace fa

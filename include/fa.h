@@ -133,8 +133,11 @@ size_t fa_fp8_workspace_size(int B, int Hq, int Hkv, int N, int d);
  * `rotation_seed` by SplitMix64, the same for Q and K) when use_rotation is
  * non-zero; Q, K, V are quantised with one float32 scale per 64-row block
  * (s = amax / 448); P is quantised per 128-key tile with V's block scale
- * folded in. Inputs are bf16; O is bf16, LSE float32. The workspace is
- * overwritten.
+ * folded in. Inputs are bf16; O is bf16, LSE float32. Only d = 128 is built
+ * (FA_ERR_UNSUPPORTED otherwise). The workspace is overwritten; afterwards it
+ * holds, each region starting on a 1024-byte boundary: e4m3 codes of Q
+ * [B*Hq, N, d], K and V [B*Hkv, N, d], then float32 block scales of Q
+ * [B*Hq, ceil(N/64)], K and V [B*Hkv, ceil(N/64)].
  */
 fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
                      uint64_t rotation_seed, int use_rotation,

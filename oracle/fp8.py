@@ -184,9 +184,12 @@ def fp8_attention_forward(q, k, v, causal: bool, scale: float, sigma=None,
     return o, lse
 
 
-def naive_fp8_attention_forward(q, k, v, causal: bool, scale: float):
+def naive_fp8_attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int = 2048, heads=None):
     """Baseline FP8: per-tensor amax scales for Q, K, V, no rotation, exact
-    softmax, normalised P rounded to e4m3. Returns O."""
+    softmax, normalised P rounded to e4m3. Returns O. Query rows are formed
+    ``row_chunk`` at a time (each row still sees all of its keys). ``heads``,
+    a list of (b, h), limits which heads' outputs are computed (the others
+    are NaN); the scales still come from the whole tensors."""
     def per_tensor(x):
         x32 = np.asarray(x, np.float64).astype(np.float32)
         amax = np.float32(np.max(np.abs(x32)))
@@ -204,15 +207,18 @@ def naive_fp8_attention_forward(q, k, v, causal: bool, scale: float):
     vscale = float(vamax / np.float32(E4M3_MAX))
     B, Hq, N, d = qh.shape
     g = Hq // kh.shape[1]
-    o = np.empty((B, Hq, N, d))
-    for b in range(B):
-        for h in range(Hq):
-            s = scale * (qh[b, h] @ kh[b, h // g].T)
-            if causal:
-                s = np.where(np.triu(np.ones((N, N), bool), 1), -np.inf, s)
-            m = np.max(s, axis=1, keepdims=True)
-            e = np.exp(s - m)
-            p = e / e.sum(axis=1, keepdims=True)
-            pq = e4m3_round(p.astype(np.float32)).astype(np.float64)
-            o[b, h] = (pq @ vvals[b, h // g]) * vscale
+    o = np.full((B, Hq, N, d), np.nan)
+    todo = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else list(heads)
+    for b, h in todo:
+        if True:
+            for r0 in range(0, N, row_chunk):
+                r1 = min(N, r0 + row_chunk)
+                s = scale * (qh[b, h, r0:r1] @ kh[b, h // g].T)
+                if causal:
+                    s = np.where(np.arange(N)[None, :] > np.arange(r0, r1)[:, None], -np.inf, s)
+                m = np.max(s, axis=1, keepdims=True)
+                e = np.exp(s - m)
+                p = e / e.sum(axis=1, keepdims=True)
+                pq = e4m3_round(p.astype(np.float32)).astype(np.float64)
+                o[b, h, r0:r1] = (pq @ vvals[b, h // g]) * vscale
     return o

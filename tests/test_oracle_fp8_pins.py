@@ -142,3 +142,18 @@ def test_naive_fp8_is_worse_with_outliers():
     rmse = lambda a: math.sqrt(np.mean((a - exact) ** 2))
     assert rmse(o_blk) < rmse(o_naive)
     assert np.linalg.norm(o_naive - exact) / np.linalg.norm(exact) < 0.3
+
+
+def test_naive_row_chunking_does_not_change_result():
+    q, k, v = _fp8_inputs(N=100, d=64, seed=13)
+    a = oracle.naive_fp8_attention_forward(q, k, v, True, 0.125, row_chunk=7)
+    b = oracle.naive_fp8_attention_forward(q, k, v, True, 0.125, row_chunk=1000)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_naive_head_subset_matches_full():
+    q, k, v = _fp8_inputs(N=80, d=64, H=3, seed=14)
+    full = oracle.naive_fp8_attention_forward(q, k, v, False, 0.125)
+    part = oracle.naive_fp8_attention_forward(q, k, v, False, 0.125, heads=[(0, 2)])
+    np.testing.assert_array_equal(part[0, 2], full[0, 2])
+    assert np.isnan(part[0, 0]).all()
