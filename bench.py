@@ -99,6 +99,24 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """The largest of every rank's x (device time is reported as the slowest
+    rank's). A no-op on one rank."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs the same per-GPU work, so the job did
+    world x steps x flops in the slowest rank's time."""
+    return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
 def _oracle_threads():
     try:
         import threadpoolctl
@@ -256,12 +274,9 @@ def run_ours(args, rank, world, local_rank):
     fwd_ms = [a.elapsed_time(b_) for a, b_, _ in ev]
     bwd_ms = [b_.elapsed_time(c) for _, b_, c in ev]
     clocks = clk.summary()
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     flops = sum((w.fwd_flops(causal) if p_ == "fwd" else w.bwd_flops(causal)) for p_ in passes)
-    value = world * flops * args.steps / (ms * 1e-3) / 1e12
+    value = weak_scaling_value(flops, args.steps, world, ms)
 
     # --- end to end through the public API with pinned host buffers: every
     # step copies its inputs host->device and reads O and LSE back
@@ -288,12 +303,8 @@ def run_ours(args, rank, world, local_rank):
                 h.copy_(t, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": weak_scaling_value(flops, e2e_steps, world, e2e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
     assert fa.fa_last_device_status() == 0
 

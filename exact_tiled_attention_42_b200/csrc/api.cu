@@ -56,9 +56,10 @@ fa_status check_shape(int B, int Hq, int Hkv, int N, int d, float scale) {
   if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  // one 1-D grid of (batch x head) x (query or key tiles): must fit in 2^31 - 1
   const long long BH = static_cast<long long>(B) * Hq;
   const long long tiles = (N + 127) / 128;
-  if (BH > 0x7fffffffLL || (tiles + 1) / 2 > 65535) return FA_ERR_UNSUPPORTED;
+  if (BH * tiles > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -180,7 +181,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
   const long long BH = static_cast<long long>(B) * Hq, BHkv = static_cast<long long>(B) * Hkv;
   const int T = (N + 127) / 128;
-  if (T > 65535 || BHkv > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;  // grid = (B*Hkv, key tiles)
+
   const size_t vec_bytes = up256(static_cast<size_t>(BH) * T * 128 * sizeof(float));
   char* ws = static_cast<char*>(workspace);
   fa::BwdParams p;

@@ -159,8 +159,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int bkv = blockIdx.x;  // b * Hkv + kvh
-  const int j = blockIdx.y;    // key tile
+  // 1-D grid, head-major: all key tiles of one KV head back to back (the
+  // longest causal loops first), so resident CTAs share a few heads' Q, dO
+  // and dQ accumulator in L2.
+  const int bkv = static_cast<int>(blockIdx.x) / p.num_tiles;  // b * Hkv + kvh
+  const int j = static_cast<int>(blockIdx.x) - bkv * p.num_tiles;  // key tile
   const int b = bkv / p.Hkv;
   const int kvh = bkv - b * p.Hkv;
   const int T = p.num_tiles;
@@ -338,13 +341,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       uint32_t pk[64];
       {
         float s[BT];
+        {
+          uint32_t t[4][32];
 #pragma unroll
-        for (int c = 0; c < BT; c += 32) {
-          uint32_t t[32];
-          tmem_ld_x32(tS + c, t);
+          for (int c = 0; c < 4; ++c) tmem_ld_x32(tS + 32 * c, t[c]);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) s[c + e] = __uint_as_float(t[e]);
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(t[c][e]);
         }
 #pragma unroll
         for (int c = 0; c < BT; c += 4) {
@@ -526,7 +531,7 @@ cudaError_t launch_main(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CU
   auto kern = bwd_bf16_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(B * p.Hkv, p.num_tiles);  // key tile j = blockIdx.y: longest causal loops launch first
+  dim3 grid(B * p.Hkv * p.num_tiles);
   kern<<<grid, BWD_THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p);
   return cudaGetLastError();
 }

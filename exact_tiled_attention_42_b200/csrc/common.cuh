@@ -238,6 +238,25 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x evaluated on the FMA pipe instead of the MUFU unit, so that a share of
+// the softmax exponentials can run beside the MUFU ones. Range reduction:
+// x = j + f with j = round-to-nearest(x) (read from the low mantissa bits of
+// x + 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose
+// coefficients were fitted for minimal maximum relative error
+// (fit_exp2_poly.py: 7.5e-5, below bf16's 2^-9 rounding of P); 2^j is added
+// to the exponent bits. Valid for x <= 64; inputs below -126 (including -inf
+// from masked scores) are clamped, giving at most 2^-125.
+__device__ __forceinline__ float exp2_poly(float x) {
+  constexpr float C0 = 0x1.fff692p-1f, C1 = 0x1.62f31ap-1f, C2 = 0x1.f0de1cp-3f, C3 = 0x1.c3f76p-5f;
+  constexpr float SHIFT = 12582912.0f;  // 1.5 * 2^23
+  x = fmaxf(x, -126.0f);
+  const float t = __fadd_rn(x, SHIFT);
+  const float f = __fsub_rn(x, __fsub_rn(t, SHIFT));
+  const float p = fmaf(fmaf(fmaf(C3, f, C2), f, C1), f, C0);
+  const uint32_t j = static_cast<uint32_t>(__float_as_int(t) - __float_as_int(SHIFT));
+  return __uint_as_float(__float_as_uint(p) + (j << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -101,8 +101,12 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int bh = blockIdx.x;  // b * Hq + hq
-  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.y);  // longest causal rows first
+  // 1-D grid: heads vary fastest and the query-tile pairs with the most key
+  // tiles (causal) come first across all heads, so the light pairs form the
+  // tail (measured faster than running each head's pairs back to back).
+  const int BH = static_cast<int>(gridDim.x) / p.num_pairs;
+  const int bh = static_cast<int>(blockIdx.x) % BH;  // b * Hq + hq
+  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
   const int b = bh / p.Hq;
   const int hq = bh - b * p.Hq;
   const int kvh = b * p.Hkv + hq / p.group;
@@ -280,13 +284,16 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       }
       tc_fence_after();
       float s[BN];
+      {
+        // all four loads in flight before the single wait
+        uint32_t r[4][32];
 #pragma unroll
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld_x32(tS + c, r);
+        for (int c = 0; c < 4; ++c) tmem_ld_x32(tS + 32 * c, r[c]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(r[i]);
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[c][i]);
       }
       const int kv0 = j * BN;
       const bool edge = (kv0 + BN > p.N) || (CAUSAL && kv0 + BN - 1 > qt * BM);
@@ -400,7 +407,7 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
   auto kern = fwd_bf16_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(BH, p.num_pairs);
+  dim3 grid(BH * p.num_pairs);
   kern<<<grid, FWD_THREADS, C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmO, p);
   return cudaGetLastError();
 }

@@ -97,8 +97,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int bh = blockIdx.x;
-  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.y);
+  // 1-D grid: heads vary fastest and the query-tile pairs with the most key
+  // tiles (causal) come first across all heads, so the light pairs form the
+  // tail (measured faster than running each head's pairs back to back).
+  const int BH = static_cast<int>(gridDim.x) / p.num_pairs;
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
   const int b = bh / p.Hq;
   const int hq = bh - b * p.Hq;
   const int kvh = b * p.Hkv + hq / p.group;
@@ -266,20 +270,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_after();
       float s[BN];
+      {
+        // all four loads in flight before the single wait
+        uint32_t r[4][32];
 #pragma unroll
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld_x32(tS + c, r);
+        for (int c = 0; c < 4; ++c) tmem_ld_x32(tS + 32 * c, r[c]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(r[i]);
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[c][i]);
       }
       const int kb0 = 2 * j;  // key blocks of this tile: 2j (keys 0-63) and 2j+1 (64-127)
       const int kb1 = min(2 * j + 1, p.nblk - 1);
+      // log2-domain score factor of each key half (folded into the FFMA
+      // before the exponential); the max is taken on raw scores per half
       const float f0 = crow * sKs[kb0], f1 = crow * sKs[kb1];
       const float w0 = sVs[kb0] * wlift, w1 = sVs[kb1] * wlift;
-#pragma unroll
-      for (int c = 0; c < BN; ++c) s[c] *= (c < 64 ? f0 : f1);
       const int kv0 = j * BN;
       const bool edge = (kv0 + BN > p.N) || (CAUSAL && kv0 + BN - 1 > qt * BM);
       if (edge) {
@@ -288,13 +295,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < BN; ++c)
           if (kv0 + c >= lim) s[c] = -INFINITY;
       }
-      float mx[8];
+      float mx[8], mlo, mhi;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = s[i];
+      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll
-      for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-      const float tile_max = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int c = 0; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+      mlo = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+#pragma unroll
+      for (int c = 64; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+      mhi = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float tile_max = fmaxf(mlo * f0, mhi * f1);
       if (j == 0) {
         m = tile_max;
       } else if (__any_sync(0xffffffffu, tile_max > m)) {
@@ -318,8 +330,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float w = i < 16 ? w0 : w1;
-        const float a0 = ex2(s[4 * i] + neg_m), a1 = ex2(s[4 * i + 1] + neg_m);
-        const float a2 = ex2(s[4 * i + 2] + neg_m), a3 = ex2(s[4 * i + 3] + neg_m);
+        const float f = i < 16 ? f0 : f1;
+        const float a0 = ex2(fmaf(s[4 * i], f, neg_m)), a1 = ex2(fmaf(s[4 * i + 1], f, neg_m));
+        const float a2 = ex2(fmaf(s[4 * i + 2], f, neg_m)), a3 = ex2(fmaf(s[4 * i + 3], f, neg_m));
         ls[i & 3] += (a0 + a1) + (a2 + a3);
         pk[i] = e4m3x4(a0 * w, a1 * w, a2 * w, a3 * w);
       }
@@ -387,7 +400,7 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
   auto kern = fwd_fp8_kernel<CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(BH, p.num_pairs);
+  dim3 grid(BH * p.num_pairs);
   kern<<<grid, THREADS, Cfg::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmO, p);
   return cudaGetLastError();
 }

@@ -70,7 +70,7 @@ def test_fwd_rejects_bad_arguments(lib):
     assert fwd(lib, scale=float("nan")) == 1
     assert fwd(lib, d=96) == 2
     assert fwd(lib, d=256) == 2
-    assert fwd(lib, N=65535 * 256 + 1) == 2
+    assert fwd(lib, B=65536, Hq=256, Hkv=256, N=16384) == 2  # grid of more than 2^31 - 1 CTAs
     assert fwd(lib, q=P + 8) == 3
     assert fwd(lib, lse=P + 4) == 3
 

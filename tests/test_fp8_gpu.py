@@ -11,9 +11,11 @@
   itself moves by the same amount (0.06 max, 3e-4 RMS on a 385-row case) when
   its scores are perturbed by 1e-4 relative. So the bound per element is
   2e-2 + 1/4 * Pmax_i * max|V| (one step on the row's two largest
-  probabilities; Pmax_i the exact largest probability of row i), the RMS of
-  kernel - emulation must stay under a tenth of the emulation's own RMS error
-  against exact attention, and LSE must agree within 1e-2.
+  probabilities; Pmax_i the exact largest probability of row i) and LSE must
+  agree within 1e-2. The RMS of kernel - emulation must stay under half the
+  emulation's own RMS error against exact attention, and the kernel's RMS
+  error against exact attention may exceed the emulation's by at most 10 %:
+  the kernel must be as accurate as the emulated method, not equal to it.
 * The kernel's error against exact fp64 attention is reported next to the
   naive per-tensor FP8 baseline's, and must not be worse.
 """
@@ -45,7 +47,9 @@ def check_against_emulation(o, lse, o_emu, lse_emu, q, k, v, causal, scale):
     assert np.all(err <= bound), f"{np.count_nonzero(err > bound)} elements past the flip bound, max {err.max()}"
     rms_diff = math.sqrt(np.mean((o - o_emu) ** 2))
     rms_emu = math.sqrt(np.mean((o_emu - exact) ** 2))
-    assert rms_diff <= 0.1 * rms_emu, (rms_diff, rms_emu)
+    rms_gpu = math.sqrt(np.mean((o - exact) ** 2))
+    assert rms_diff <= 0.5 * rms_emu, (rms_diff, rms_emu)
+    assert rms_gpu <= 1.1 * rms_emu + 1e-4, (rms_gpu, rms_emu)
     assert np.max(np.abs(lse - lse_emu)) <= FP8_LSE_MAX_ABS, np.max(np.abs(lse - lse_emu))
     return exact
 
