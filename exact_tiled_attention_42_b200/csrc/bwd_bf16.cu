@@ -26,7 +26,9 @@
 // accumulator with TMA reduce-add (thread = query row); warp 8 loads with TMA;
 // one thread of warp 9 issues every MMA. P^T and dS^T (bf16) are written over
 // the S^T columns; for d = 128 the dQ accumulator reuses the dP^T columns and
-// dS reuses the shared-memory slot of dO_i once dV has read it.
+// dS reuses the shared-memory slot of dO_i once dV has read it. dK is issued
+// as soon as dS^T is in tensor memory, before dS has reached shared memory
+// (which waits for dV), and dQ once it has.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -54,7 +56,7 @@ struct BwdCfg {
   static constexpr int OFF_STG = OFF_DS + (DS_ALIAS ? 0 : DS_BYTES);  // 4 warps x 2 buffers x 2 KB
   static constexpr int OFF_VEC = OFF_STG + 16384;  // 2 slots x (-LSE log2e, D) x 512 B
   static constexpr int OFF_BAR = OFF_VEC + 2048;
-  static constexpr int NUM_BARS = 19;
+  static constexpr int NUM_BARS = 20;
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
   static constexpr uint32_t COL_S = 0;    // S^T; then P^T bf16 in [0,64) and dS^T bf16 in [64,128)
   static constexpr uint32_t COL_DP = 128;
@@ -76,7 +78,8 @@ struct BwdBars {
   __device__ uint32_t s_full() const { return base + 8u * 9; }
   __device__ uint32_t dp_full() const { return base + 8u * 10; }
   __device__ uint32_t p_ready() const { return base + 8u * 11; }
-  __device__ uint32_t ds_ready() const { return base + 8u * 12; }
+  __device__ uint32_t dst_ready() const { return base + 8u * 12; }  // dS^T in tensor memory
+  __device__ uint32_t dss_ready() const { return base + 8u * 19; }  // dS in shared memory
   __device__ uint32_t dv_done() const { return base + 8u * 13; }
   __device__ uint32_t dq_full() const { return base + 8u * 14; }
   __device__ uint32_t dq_free() const { return base + 8u * 15; }
@@ -186,7 +189,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(bars.s_full(), 1);
     mbar_init(bars.dp_full(), 1);
     mbar_init(bars.p_ready(), 4);
-    mbar_init(bars.ds_ready(), 4);
+    mbar_init(bars.dst_ready(), 4);
+    mbar_init(bars.dss_ready(), 4);
     mbar_init(bars.dv_done(), 1);
     mbar_init(bars.dq_full(), 1);
     mbar_init(bars.dq_free(), 4);
@@ -299,13 +303,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, smem_desc_sw128(sdO + kk * 2048, C::BOX_BYTES, 1024),
                  IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bars.dv_done());
-        if (!mbar_wait(bars.ds_ready(), it & 1, abort, p.status, SITE_BWD + 8)) break;
+        if (!mbar_wait(bars.dst_ready(), it & 1, abort, p.status, SITE_BWD + 8)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)  // dK += dS^T Q_i
           mma_ts(tmem + C::COL_DK, tmem + C::COL_S + 64 + kk * 8, smem_desc_sw128(sQ + kk * 2048, C::BOX_BYTES, 1024),
                  IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bars.q_empty(st));
+        if (!mbar_wait(bars.dss_ready(), it & 1, abort, p.status, SITE_BWD + 16)) break;
         if (!C::DQ_SHARES_DP && it > 0 &&
             !mbar_wait(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
           break;
@@ -386,38 +391,46 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (lane == 0) mbar_arrive(bars.p_ready());
 
       ok = __all_sync(0xffffffffu, mbar_wait(bars.dp_full(), it & 1, abort, p.status, SITE_BWD + 11));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.dv_done(), it & 1, abort, p.status, SITE_BWD + 12));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t sdS = ds_smem(st);
+      // dS = P (dP - D): into tensor memory first (dK can start at once), then
+      // into shared memory once dV has finished reading this dO slot (dQ)
+      uint32_t dsk[64];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t t[32];
         tmem_ld_x32(tDP + cc * 32, t);
         tmem_wait_ld();
-        uint32_t dsk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c = cc * 32 + 2 * e;
           const float2 dd = *reinterpret_cast<const float2*>(vec_d + c);
           const uint32_t pp = pk[cc * 16 + e];
-          dsk[e] = pack_bf16x2(bf16_lo(pp) * (__uint_as_float(t[2 * e]) - dd.x),
-                               bf16_hi(pp) * (__uint_as_float(t[2 * e + 1]) - dd.y));
+          dsk[cc * 16 + e] = pack_bf16x2(bf16_lo(pp) * (__uint_as_float(t[2 * e]) - dd.x),
+                                         bf16_hi(pp) * (__uint_as_float(t[2 * e + 1]) - dd.y));
         }
-        tmem_st_x16(tS + 64 + cc * 16, dsk);
+        tmem_st_x16(tS + 64 + cc * 16, *reinterpret_cast<const uint32_t(*)[16]>(dsk + cc * 16));
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.dst_ready());
+      ok = __all_sync(0xffffffffu, mbar_wait(bars.dv_done(), it & 1, abort, p.status, SITE_BWD + 12));
+      if (!ok) break;
+      const uint32_t sdS = ds_smem(st);
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint32_t addr = sdS + (cc >> 1) * C::BOX_BYTES + sw128_offset(r, (cc & 1) * 4 + q);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dsk[4 * q]), "r"(dsk[4 * q + 1]),
-                       "r"(dsk[4 * q + 2]), "r"(dsk[4 * q + 3])
+          const int e = cc * 16 + 4 * q;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dsk[e]), "r"(dsk[e + 1]),
+                       "r"(dsk[e + 2]), "r"(dsk[e + 3])
                        : "memory");
         }
-      }
-      tmem_wait_st();
       fence_proxy_async_smem();
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars.ds_ready());
+      if (lane == 0) mbar_arrive(bars.dss_ready());
     }
     // ------------------------------------------------------------ dK, dV epilogue
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.dkdv_done(), 0, abort, p.status, SITE_BWD + 13));
