@@ -99,6 +99,39 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "roofline_traffic.md")
+
+
+def sources_sha256(paths) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(key: str):
+    """DRAM bytes per launch measured by ncu for `key`, from the table in
+    profiles/roofline_traffic.md, or None when there is no row for it or the
+    kernel sources have changed since the counters were taken (the row keeps
+    the sha256 of the sources it was measured on)."""
+    try:
+        rows = [r for r in open(TRAFFIC_TABLE).read().splitlines() if r.startswith("| ") and "|" in r[2:]]
+    except OSError:
+        return None
+    for r in rows:
+        cells = [c.strip() for c in r.strip().strip("|").split("|")]
+        if len(cells) < 4 or cells[0] != key:
+            continue
+        try:
+            if sources_sha256(cells[1].split()) == cells[2]:
+                return float(cells[3])
+        except (OSError, ValueError):
+            return None
+    return None
+
+
 def max_over_ranks(x: float, world: int, device="cuda") -> float:
     """The largest of every rank's x (device time is reported as the slowest
     rank's). A no-op on one rank."""
@@ -322,8 +355,10 @@ def run_ours(args, rank, world, local_rank):
     # figure is a lower bound for the main kernel alone
     if "bwd" in passes:
         dom, achieved = "fa_bwd: bwd_pre_kernel + bwd_bf16_kernel + bwd_post_kernel", bwd_tf
+        traffic = recorded_traffic(f"fa_bwd {args.workload}")
     else:
         dom, achieved = "fwd_bf16_kernel", fwd_tf
+        traffic = recorded_traffic(f"fwd_bf16_kernel {args.workload}")
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         v, el, heads, threads = cpu_oracle_sample(w, causal, passes, seconds_budget=args.cpu_seconds)
@@ -340,7 +375,8 @@ def run_ours(args, rank, world, local_rank):
         "bwd_tflops": bwd_tf, "bwd_frac_of_peak": (bwd_tf / peak) if bwd_tf else None,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                      "peak_kind": f"{pk_kind} bf16 dense, sustained (kernel timed inside a long loop)",
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None},
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "fp8": fp8,
