@@ -343,47 +343,46 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_after();
       const float* vec_lse = reinterpret_cast<const float*>(base_ptr + C::OFF_VEC + st * 1024);
       const float* vec_d = vec_lse + 128;
-      uint32_t pk[64];
-      {
-        float s[BT];
-        {
-          uint32_t t[4][32];
+      // P^T in two halves of 64 queries (keeps the live registers low): the
+      // packed bf16 P^T of queries 64h.. lands in columns 32h.. of S^T, which
+      // this thread has already read
+      const int qlim = p.N - i * BT;  // queries past N are padding
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld_x32(tS + 32 * c, t[c]);
+      for (int h = 0; h < 2; ++h) {
+        float s[64];
+        {
+          uint32_t t[2][32];
+          tmem_ld_x32(tS + 64 * h, t[0]);
+          tmem_ld_x32(tS + 64 * h + 32, t[1]);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(t[c][e]);
         }
 #pragma unroll
-        for (int c = 0; c < BT; c += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(vec_lse + c);
+        for (int c = 0; c < 64; c += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(vec_lse + 64 * h + c);
           s[c] = ex2(fmaf(s[c], cl2, l4.x));
           s[c + 1] = ex2(fmaf(s[c + 1], cl2, l4.y));
           s[c + 2] = ex2(fmaf(s[c + 2], cl2, l4.z));
           s[c + 3] = ex2(fmaf(s[c + 3], cl2, l4.w));
         }
-        if (CAUSAL && i == j) {  // diagonal tile: key r sees queries c >= r
+        if (CAUSAL && i == j) {  // diagonal tile: key r sees queries >= r
 #pragma unroll
-          for (int c = 0; c < BT; ++c)
-            if (c < r) s[c] = 0.f;
+          for (int c = 0; c < 64; ++c)
+            if (64 * h + c < r) s[c] = 0.f;
         }
-        const int qlim = p.N - i * BT;  // queries past N are padding
         if (qlim < BT) {
 #pragma unroll
-          for (int c = 0; c < BT; ++c)
-            if (c >= qlim) s[c] = 0.f;
+          for (int c = 0; c < 64; ++c)
+            if (64 * h + c >= qlim) s[c] = 0.f;
         }
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) pk[e] = pack_bf16x2(s[2 * e], s[2 * e + 1]);
-      }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t t[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) t[e] = pk[c * 16 + e];
-        tmem_st_x16(tS + c * 16, t);
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[2 * e], s[2 * e + 1]);
+        tmem_st_x16(tS + 32 * h, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+        tmem_st_x16(tS + 32 * h + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -393,21 +392,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bars.dp_full(), it & 1, abort, p.status, SITE_BWD + 11));
       if (!ok) break;
       tc_fence_after();
-      // dS = P (dP - D): into tensor memory first (dK can start at once), then
-      // into shared memory once dV has finished reading this dO slot (dQ)
+      // dS = P (dP - D), 32 queries at a time with P^T read back from tensor
+      // memory: into tensor memory first (dK can start at once), then into
+      // shared memory once dV has finished reading this dO slot (dQ)
       uint32_t dsk[64];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t t[32];
+        uint32_t t[32], pp[16];
         tmem_ld_x32(tDP + cc * 32, t);
+        tmem_ld_x16(tS + cc * 16, pp);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c = cc * 32 + 2 * e;
           const float2 dd = *reinterpret_cast<const float2*>(vec_d + c);
-          const uint32_t pp = pk[cc * 16 + e];
-          dsk[cc * 16 + e] = pack_bf16x2(bf16_lo(pp) * (__uint_as_float(t[2 * e]) - dd.x),
-                                         bf16_hi(pp) * (__uint_as_float(t[2 * e + 1]) - dd.y));
+          dsk[cc * 16 + e] = pack_bf16x2(bf16_lo(pp[e]) * (__uint_as_float(t[2 * e]) - dd.x),
+                                         bf16_hi(pp[e]) * (__uint_as_float(t[2 * e + 1]) - dd.y));
         }
         tmem_st_x16(tS + 64 + cc * 16, *reinterpret_cast<const uint32_t(*)[16]>(dsk + cc * 16));
       }
