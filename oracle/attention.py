@@ -22,7 +22,9 @@ Readings where the pages are silent (the method's definition is fixed by the
 workload statement, not by the pages): scale multiplies Q K^T; the causal mask
 keeps key j for query i iff j <= i; LSE is the natural log of the row's sum of
 exp(scale * S); the backward is the analytic gradient of O with respect to Q,
-K and V (dK and dV summed over the query heads sharing a KV head).
+K and V (dK and dV summed over the query heads sharing a KV head). For fewer
+query rows than keys (Nq < Nk, decoding against a cache) the forward treats
+the queries as the last Nq positions: query i keeps keys j <= i + Nk - Nq.
 
 Inputs are float arrays [B, H, N, d] (Q and dO with Hq heads, K and V with Hkv
 heads); every computation runs in float64.
@@ -45,10 +47,12 @@ def _heads(q, k):
 
 def _scores(qh, kh, scale, causal, row0, row1):
     """Rows row0..row1-1 of S = scale * Q K^T, with -inf where the causal mask
-    removes a key."""
+    removes a key. With Nq query rows and Nk >= Nq keys, query i sits at key
+    position i + Nk - Nq (the queries are the last Nq positions of the
+    sequence, as when decoding against a cache); with Nq = Nk this is j <= i."""
     s = scale * (qh[row0:row1] @ kh.T)
     if causal:
-        i = np.arange(row0, row1)[:, None]
+        i = np.arange(row0, row1)[:, None] + (kh.shape[0] - qh.shape[0])
         j = np.arange(kh.shape[0])[None, :]
         s = np.where(j > i, -np.inf, s)
     return s

@@ -230,3 +230,28 @@ def test_online_softmax_large_scores_with_stale_max():
     o2, l2 = oracle.online_softmax_forward(q, k, v, False, 1.0, 8, 8.0)
     np.testing.assert_allclose(o2, o1, atol=1e-12)
     np.testing.assert_allclose(l2, l1, rtol=1e-13)
+
+
+# --- fewer query rows than keys ------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_query_suffix_equals_rows_of_square_problem(causal):
+    """Nq < Nk: the last Nq queries of a square problem, run alone against all
+    Nk keys, give exactly those rows of the square result (the causal mask is
+    aligned to the end of the key sequence)."""
+    q, k, v = _rand((2, 4, 40, 8), 40), _rand((2, 2, 40, 8), 41), _rand((2, 2, 40, 8), 42)
+    full_o, full_l = oracle.attention_forward(q, k, v, causal, 0.3)
+    for nq in (1, 3, 17, 40):
+        o, l = oracle.attention_forward(q[:, :, 40 - nq:], k, v, causal, 0.3)
+        np.testing.assert_allclose(o, full_o[:, :, 40 - nq:], atol=1e-14)
+        np.testing.assert_allclose(l, full_l[:, :, 40 - nq:], atol=1e-14)
+
+
+def test_single_query_uniform_scores():
+    """One query with Q = 0 against Nk keys: O is the mean of all V rows and
+    LSE = log Nk, causal or not (the query is the last position)."""
+    k, v = _rand((1, 1, 25, 8), 43), _rand((1, 1, 25, 8), 44)
+    for causal in (False, True):
+        o, l = oracle.attention_forward(np.zeros((1, 1, 1, 8)), k, v, causal, 0.7)
+        np.testing.assert_allclose(o[0, 0, 0], v[0, 0].mean(0), atol=1e-14)
+        assert abs(l[0, 0, 0] - math.log(25)) < 1e-14
