@@ -342,6 +342,7 @@ def run_ours(args, rank, world, local_rank):
     assert fa.fa_last_device_status() == 0
 
     fp8 = None if args.no_fp8 else run_fp8_leg(args, fa, stream)
+    decode = None if args.no_decode else run_decode_leg(args, fa, stream)
     assert fa.fa_last_device_status() == 0
 
     if rank != 0:
@@ -380,6 +381,7 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "fp8": fp8,
+        "decode": decode,
         "gpu_launches": args.steps * (1 + (3 if "bwd" in passes else 0)),
         "clocks": clocks,
     }
@@ -424,6 +426,46 @@ def run_fp8_leg(args, fa, stream):
             "includes": "quantisation pre-pass (Hadamard rotation, 64-row block scales) + FP8 forward"}
 
 
+def run_decode_leg(args, fa, stream):
+    """Decode step (one query row per head against a 16K-key cache, GQA 32/8),
+    timed with events around each fa_fwd_decode call (split pass + combine).
+    HBM-bound: reported in GB/s of algorithmic bytes (K, V, Q read; O, LSE
+    written) against the measured copy bandwidth. K and V (1.07 GB) exceed L2."""
+    import torch
+    w = WORKLOADS["decode"]
+    causal = w.causal[0]
+    kv = attention_inputs(w.B, w.Hkv, w.Hkv, w.N, w.d, w.seed, with_dout=False)
+    qq = attention_inputs(w.B, w.Hq, w.Hq, w.nq, w.d, w.seed + 1000, with_dout=False)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    q, k, v = to_dev(qq["q"]), to_dev(kv["k"]), to_dev(kv["v"])
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.nq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(fa.fa_decode_workspace_size(w.B, w.Hq, w.Hkv, w.nq, w.N, w.d, 0), dtype=torch.uint8,
+                     device="cuda")
+
+    def call():
+        fa.fa_fwd_decode(q, k, v, causal=causal, out=o, lse=lse, workspace=ws)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 500))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b_ in ev:
+        a.record(stream)
+        call()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b_) for a, b_ in ev)
+    nbytes = (k.numel() + v.numel() + q.numel() + o.numel()) * 2 + lse.numel() * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    pk, pk_kind = peaks()
+    return {"workload": f"decode: B={w.B} Hq={w.Hq} Hkv={w.Hkv} Nq={w.nq} Nk={w.N} d={w.d} causal={causal}",
+            "gbs": gbs, "us_per_call": ms * 1e3, "calls": steps, "bytes_per_call": nbytes,
+            "peak_gbs": pk["hbm_gbs"], "peak_kind": f"{pk_kind} HBM copy bandwidth", "frac_of_peak": gbs / pk["hbm_gbs"],
+            "includes": "split pass over the keys + log-sum-exp combine"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -434,7 +476,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward leg")
-    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(WORKLOADS),
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode (split-KV) leg")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(k for k, v in WORKLOADS.items() if not v.nq),
                     help="workload to run (profiling of other shapes; the headline is the default)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -13,6 +13,8 @@ from .api import (  # noqa: F401
     fa_bwd,
     fa_bwd_noalloc,
     fa_fwd_fp8,
+    fa_fwd_decode,
+    fa_decode_workspace_size,
     fa_bwd_workspace_size,
     fa_fp8_workspace_size,
     fa_status_string,

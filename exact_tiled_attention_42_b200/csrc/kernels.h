@@ -82,4 +82,29 @@ cudaError_t launch_fp8_quant(const Fp8Params& p, cudaStream_t stream);
 cudaError_t launch_fwd_fp8(const CUtensorMap& tmQ8, const CUtensorMap& tmK8, const CUtensorMap& tmV8,
                            const CUtensorMap& tmO, const Fp8Params& p, int BH, bool causal, cudaStream_t stream);
 
+struct DecParams {
+  const uint16_t* q;  // bf16 [B*Hq, Nq, d]
+  uint16_t* o;        // bf16 [B*Hq, Nq, d]
+  float* lse;         // [B*Hq, Nq]
+  float* o_part;      // workspace [B*Hkv, splits, R, d] fp32, normalised within the split
+  float* lse_part;    // workspace [B*Hkv, splits, R], natural log (-inf: no key in the split)
+  int* status;
+  int Hq;
+  int Hkv;
+  int group;          // Hq / Hkv
+  int Nq;
+  int Nk;
+  int R;              // group * Nq query rows per KV head
+  int splits;
+  int keys_per_split; // multiple of 64
+  int causal;
+  float scale_log2;
+};
+
+// Decode-shaped forward: split pass over key chunks (one CTA per KV head and
+// split) then the LSE-weighted combine. tmK/tmV: bf16 [B*Hkv, Nk, d], 64 x 64
+// boxes, 128B swizzle.
+cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecParams& p, int B, int d,
+                          cudaStream_t stream);
+
 }  // namespace fa

@@ -145,6 +145,38 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
                      int B, int Hq, int Hkv, int N, int d, int causal, float scale,
                      cudaStream_t stream);
 
+/*
+ * Bytes of device workspace fa_fwd_decode needs for these sizes and
+ * num_splits (0 = automatic, as in fa_fwd_decode): per KV head, split and
+ * query row, one float32 partial output row and one float32 log-sum-exp.
+ * Returns 0 for invalid or unsupported sizes.
+ */
+size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits);
+
+/*
+ * Forward for few query rows against a long key sequence (decoding with a
+ * key/value cache): q, o are [B, Hq, Nq, d] bf16, k, v [B, Hkv, Nk, d] bf16,
+ * lse [B, Hq, Nq] float32 (natural log). The computation is fa_fwd's with
+ * Nq rows: "FlashAttention: The Algorithm That Made Long-Context AI
+ * Possible" (sections "The quadratic bottleneck in standard attention" and
+ * "What tiling changes"); the pages do not discuss decoding. With causal
+ * non-zero the queries are the last Nq positions of the sequence: query i
+ * keeps keys j <= i + Nk - Nq (requires Nk >= Nq).
+ * The key sequence is split into num_splits chunks processed by separate
+ * CTAs (0 = choose automatically: enough CTAs to fill the GPU, at least 256
+ * keys each); their partial outputs, written to the workspace, are merged by
+ * log-sum-exp. Supported: d = 64 or 128, and (Hq / Hkv) * Nq <= 16 query rows
+ * per KV head (FA_ERR_UNSUPPORTED otherwise). causal with Nk < Nq is
+ * FA_ERR_INVALID_ARG. `workspace` is device memory of at least
+ * fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits) bytes,
+ * 16-byte aligned (FA_ERR_WORKSPACE / FA_ERR_MISALIGNED otherwise); it is
+ * overwritten. Two kernels run on `stream`: the split pass, then the merge.
+ */
+fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                        void* workspace, size_t workspace_bytes,
+                        int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                        int num_splits, cudaStream_t stream);
+
 /* Human-readable name of a status code (static storage, never null). */
 const char* fa_status_string(fa_status s);
 

@@ -22,6 +22,7 @@ class Workload:
     fp8: bool = False
     outlier_rate: float = 0.0
     seed: int = 42
+    nq: int = 0  # query rows when fewer than N (decoding against a cache); 0 = N
     notes: str = field(default="", compare=False)
 
     @property
@@ -50,4 +51,8 @@ WORKLOADS = {
     "fp8": Workload("fp8", 1, 16, 16, 16384, 128, (False,), passes=("fwd",), fp8=True,
                     outlier_rate=0.001, seed=46,
                     notes="FP8 e4m3 forward with outliers, 64xd block scales, Hadamard rotation"),
+    # not one of the five: one decode step (a query row per head) against a
+    # 16K-token cache, GQA 32/8
+    "decode": Workload("decode", 16, 32, 8, 16384, 128, (True,), passes=("fwd",), seed=47, nq=1,
+                       notes="decode step: 1 query row per head, 16384-key cache, GQA 4:1"),
 }

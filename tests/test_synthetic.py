@@ -57,4 +57,4 @@ def test_workloads_flop_counts():
     w = WORKLOADS["long128"]
     assert w.fwd_flops(True) == 4 * 2 * 16 * 8192 ** 2 * 128 / 2
     assert w.bwd_flops(True) == 2.5 * w.fwd_flops(True)
-    assert [w.seed for w in WORKLOADS.values()] == [42, 43, 44, 45, 46]
+    assert [w.seed for w in WORKLOADS.values()] == [42, 43, 44, 45, 46, 47]
