@@ -162,14 +162,15 @@ def fa_fwd_fp8(q, k, v, causal: bool = False, scale: float | None = None, rotati
     return out, lse
 
 
-def fa_decode_workspace_size(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, num_splits: int = 0) -> int:
-    return int(_lib.load().fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits))
+def fa_decode_workspace_size(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, num_ctas: int = 0) -> int:
+    return int(_lib.load().fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_ctas))
 
 
-def fa_fwd_decode(q, k, v, causal: bool = False, scale: float | None = None, num_splits: int = 0,
+def fa_fwd_decode(q, k, v, causal: bool = False, scale: float | None = None, num_ctas: int = 0,
                   out=None, lse=None, workspace=None, stream=None):
-    """O, LSE for Nq query rows [B,Hq,Nq,d] against k/v [B,Hkv,Nk,d] (bf16),
-    with the key sequence split across CTAs and merged by log-sum-exp."""
+    """O, LSE for Nq query rows [B,Hq,Nq,d] against k/v [B,Hkv,Nk,d] (bf16).
+    The (KV head, key tile) pairs are shared evenly by ``num_ctas`` CTAs (0 =
+    as many as fit on the GPU) and the partial results merged by log-sum-exp."""
     if q.dim() != 4 or k.dim() != 4:
         raise ValueError("q and k must be [B, H, N, d]")
     B, Hq, Nq, d = q.shape
@@ -184,11 +185,11 @@ def fa_fwd_decode(q, k, v, causal: bool = False, scale: float | None = None, num
     _check("out", out, torch.bfloat16, (B, Hq, Nq, d))
     _check("lse", lse, torch.float32, (B, Hq, Nq))
     if workspace is None:
-        n = fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits)
+        n = fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_ctas)
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
     st = _lib.load().fa_fwd_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                   B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), float(scale), int(num_splits),
+                                   B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), float(scale), int(num_ctas),
                                    _stream(stream))
     if st != FA_OK:
         raise FAError("fa_fwd_decode", st)

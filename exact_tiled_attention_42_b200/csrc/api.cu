@@ -109,23 +109,17 @@ bool make_map_e4m3(CUtensorMap* m, const void* ptr, int d, int N, long long oute
   return r == CUDA_SUCCESS;
 }
 
-// Number of key splits for the decode path: about four waves of CTAs (two
-// fit on an SM), but at least 256 keys per split; then trimmed so no split is
-// empty.
-int decode_splits(int B, int Hkv, int Nk, int requested, int* keys_per_split) {
-  long long want = requested;
-  if (want <= 0) {
-    const long long heads = static_cast<long long>(B) * Hkv;
-    want = (4 * 2 * 148 + heads - 1) / heads;
-    const long long cap = (Nk + 255) / 256;
-    if (want > cap) want = cap;
-  }
-  if (want < 1) want = 1;
-  if (want > Nk) want = Nk;
-  int kps = static_cast<int>((Nk + want - 1) / want);
-  kps = (kps + 63) / 64 * 64;
-  *keys_per_split = kps;
-  return (Nk + kps - 1) / kps;
+// Decode path: work units are (KV head, 64-key tile). Without a request the
+// split pass runs as many CTAs as fit on the device at once, never more than
+// the units or FA_DECODE_MAX_AUTO_CTAS (the bound the workspace is sized for).
+constexpr long long FA_DECODE_MAX_AUTO_CTAS = 1024;
+
+long long decode_units(int B, int Hkv, int Nk) { return static_cast<long long>(B) * Hkv * ((Nk + 63) / 64); }
+
+// CTAs the workspace must cover (device independent)
+long long decode_ctas_bound(long long units, int requested) {
+  const long long want = requested > 0 ? requested : FA_DECODE_MAX_AUTO_CTAS;
+  return want < units ? want : units;
 }
 
 }  // namespace
@@ -232,52 +226,60 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
+size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_ctas) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || num_ctas < 0 || (d != 64 && d != 128))
+    return 0;
   const int R = (Hq / Hkv) * Nq;
   if (R > 16) return 0;
-  int kps = 0;
-  const int splits = decode_splits(B, Hkv, Nk, num_splits, &kps);
-  const size_t rows = static_cast<size_t>(B) * Hkv * splits * R;
+  const long long units = decode_units(B, Hkv, Nk);
+  const size_t slots = static_cast<size_t>(decode_ctas_bound(units, num_ctas) + static_cast<long long>(B) * Hkv);
+  const size_t rows = slots * R;
   return up256(rows * d * sizeof(float)) + up256(rows * sizeof(float));
 }
 
 fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
                         size_t workspace_bytes, int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
-                        float scale, int num_splits, cudaStream_t stream) {
+                        float scale, int num_ctas, cudaStream_t stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || num_ctas < 0) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (causal && Nk < Nq) return FA_ERR_INVALID_ARG;  // a query row would see no key
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if ((Hq / Hkv) * Nq > 16) return FA_ERR_UNSUPPORTED;  // query rows per KV head
+  const long long BHkv = static_cast<long long>(B) * Hkv;
+  const long long units = decode_units(B, Hkv, Nk);
+  if (BHkv > 0x7fffffffLL || units > 0x7fffffffLL || static_cast<long long>(B) * Hq * Nq * 32 > 0x7fffffffLL)
+    return FA_ERR_UNSUPPORTED;
   const void* ptrs[] = {q, k, v, o, lse};
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
-  const size_t need = fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits);
+  const size_t need = fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_ctas);
   if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
-  int kps = 0;
-  const int splits = decode_splits(B, Hkv, Nk, num_splits, &kps);
-  const long long BHkv = static_cast<long long>(B) * Hkv;
-  if (BHkv * splits > 0x7fffffffLL || static_cast<long long>(B) * Hq * Nq * 32 > 0x7fffffffLL)
-    return FA_ERR_UNSUPPORTED;
+  long long ctas = decode_ctas_bound(units, num_ctas);
+  if (num_ctas == 0) {
+    const int fit = fa::decode_resident_ctas(d);
+    if (fit < 1) return FA_ERR_CUDA;
+    if (fit < ctas) ctas = fit;
+  }
   fa::DecParams p;
   p.q = static_cast<const uint16_t*>(q);
   p.o = static_cast<uint16_t*>(o);
   p.lse = lse;
   p.R = (Hq / Hkv) * Nq;
-  const size_t rows = static_cast<size_t>(BHkv) * splits * p.R;
+  // slots as sized by the workspace query; the kernels use the first ctas + B*Hkv
+  const size_t slots = static_cast<size_t>(decode_ctas_bound(units, num_ctas) + BHkv);
   p.o_part = static_cast<float*>(workspace);
-  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + up256(rows * d * sizeof(float)));
+  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + up256(slots * p.R * d * sizeof(float)));
   p.status = status_ptr();
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.group = Hq / Hkv;
   p.Nq = Nq;
   p.Nk = Nk;
-  p.splits = splits;
-  p.keys_per_split = kps;
+  p.tiles = (Nk + 63) / 64;
+  p.ctas = static_cast<int>(ctas);
+  p.units = units;
   p.causal = causal != 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   if (!p.status) return FA_ERR_CUDA;

@@ -7,20 +7,33 @@
 // queries taken as the last Nq positions of the sequence for the causal mask.
 // Each key and value is read once and used by only g * Nq query rows, so the
 // kernel is bound by HBM bandwidth: what matters is keeping bytes in flight on
-// every SM and spending little shared-memory bandwidth per byte. The key
-// dimension is split across CTAs (one CTA per KV head and key chunk, so the g
-// query heads of a GQA group share each K/V tile); each CTA streams its chunk
-// through a 3-stage TMA ring (two CTAs per SM) and keeps a running max and sum
-// per query row; a second kernel merges the chunks by log-sum-exp.
+// every SM and spending little shared-memory bandwidth per byte.
+//
+// Work split. The work is a list of units (KV head, 64-key tile), head-major.
+// The split pass runs as many CTAs as fit on the GPU at once (two per SM) and
+// gives CTA c the contiguous units [c*U/G, (c+1)*U/G): every CTA streams the
+// same number of tiles, whatever the number of heads or keys, and its TMA ring
+// runs on across head boundaries. A CTA writes one partial result (rows
+// normalised within its key range, plus their log-sum-exp) for each KV head it
+// touches; the g query heads of a GQA group share each K/V tile. A second
+// kernel merges the partials of a head by log-sum-exp.
 //
 // The query rows of a KV head (at most 16) form the M = 16 side of warp-level
 // bf16 MMAs (mma.sync m16n8k16, fp32 accumulate): the products are tiny dense
-// contractions and the fragments come straight from the swizzled TMA tiles
-// with ldmatrix, so shared memory is read about once per byte. Per 64-key tile
-// (8 warps):
-//   S = Q K^T  warp w: keys 8w..8w+7, all of d (Q fragments stay in registers)
-//   softmax    warp w: rows 2w, 2w+1 (two keys per lane), P (bf16) to smem
-//   O += P V   warp w: output columns 16w.. (d = 128) or 8w.. (d = 64)
+// contractions, and the K and V fragments come straight from the swizzled TMA
+// tiles with ldmatrix. One producer warp streams 64-key tiles of K and V
+// through an mbarrier ring; each of the four consumer warps owns 16 keys of
+// every tile and runs the whole tile step on its own, with no CTA barrier:
+//   S = Q K^T   16 rows x 16 keys, Q fragments held in registers
+//   softmax     running max and sum per row over the warp's keys; O rescaled
+//               only when a max grows; P stays in registers, where the S
+//               accumulator layout is already the A-operand layout of P V
+//   O += P V    16 rows x d, fp32 in registers
+// then frees the stage. When the CTA's range of a KV head ends, the four
+// warps' (max, sum, O) are merged through the stage buffer they just read.
+
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,25 +41,24 @@ namespace fa {
 namespace {
 
 constexpr int KT = 64;        // keys per tile
-constexpr int NSTAGE = 3;     // tiles in flight per CTA (two CTAs fit on an SM)
-constexpr int THREADS = 256;
+constexpr int NCW = 4;        // consumer warps; warp w owns keys 16w .. 16w + 15 of every tile
+constexpr int THREADS = (NCW + 1) * 32;  // + one producer warp
 constexpr int MR = 16;        // MMA rows: query rows of a KV head, padded
-constexpr int SS = KT + 4;    // fp32 score row stride (words)
-constexpr int PS = KT + 8;    // bf16 P row stride (elements): 144 B rows keep ldmatrix conflict-free
 constexpr float LN2 = 0.69314718055994530942f;
 
 template <int D>
 struct DecCfg {
-  static constexpr int BOX = KT * 128;          // 64 keys x 64 bf16 (128 B rows)
-  static constexpr int TILE = (D / 64) * BOX;   // one K or V tile
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = NSTAGE * TILE;
-  static constexpr int OFF_S = 2 * NSTAGE * TILE;           // fp32 [MR][SS]
-  static constexpr int OFF_P = OFF_S + MR * SS * 4;         // bf16 [MR][PS]
-  static constexpr int OFF_A = OFF_P + MR * PS * 2;         // fp32 [MR] rescale, then 1 / l
-  static constexpr int OFF_BAR = OFF_A + MR * 4;
-  static constexpr int SMEM = OFF_BAR + NSTAGE * 8 + 8 + 1024;
-  static constexpr int NB = D / 64;                         // 8-column blocks per warp in P V
+  static constexpr int NSTAGE = D == 128 ? 3 : 4;    // tiles in flight per CTA
+  static constexpr int MIN_CTAS = D == 128 ? 2 : 3;  // CTAs per SM the shared memory allows
+  static constexpr int BOX = KT * 128;               // 64 keys x 64 bf16 (128 B rows)
+  static constexpr int TILE = (D / 64) * BOX;        // one K or V tile
+  static constexpr int STAGE = 2 * TILE;             // K then V; also holds the NCW x MR x D fp32 partials
+  static constexpr int OFF_ML = NSTAGE * STAGE;      // fp32 [NCW][MR][2]: per-warp row max and sum
+  static constexpr int OFF_BAR = OFF_ML + NCW * MR * 2 * 4;
+  // barriers: full[NSTAGE], empty[NSTAGE], gather, combine; then the abort flag
+  static constexpr int NBAR = 2 * NSTAGE + 2;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 8 + 1024;
+  static_assert(NCW * MR * D * 4 == STAGE, "a stage holds the warps' partial outputs");
 };
 
 // Byte offset of element (row, col) in a tile of 64-row, 128B-swizzled boxes.
@@ -77,207 +89,252 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
 }
 
 template <int D>
-__global__ void __launch_bounds__(THREADS, 2)
+__global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const DecParams p) {
   using C = DecCfg<D>;
+  constexpr int NST = C::NSTAGE;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* const bp = smem_raw + (base - raw);
-  float* const ssc = reinterpret_cast<float*>(bp + C::OFF_S);
-  uint16_t* const sp = reinterpret_cast<uint16_t*>(bp + C::OFF_P);
-  float* const salpha = reinterpret_cast<float*>(bp + C::OFF_A);
-  volatile int* const abort = reinterpret_cast<volatile int*>(bp + C::OFF_BAR + NSTAGE * 8);
+  float* const sml = reinterpret_cast<float*>(bp + C::OFF_ML);
+  const uint32_t bar_full = base + C::OFF_BAR;
+  const uint32_t bar_empty = bar_full + 8 * NST;
+  const uint32_t bar_gather = bar_empty + 8 * NST;  // every warp has finished reading the stage
+  const uint32_t bar_comb = bar_gather + 8;         // every warp's partial is in the stage
+  volatile int* const abort = reinterpret_cast<volatile int*>(bp + C::OFF_BAR + C::NBAR * 8);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g4 = lane >> 2, t4 = lane & 3;  // mma fragment row group and column pair
 
-  const int bkv = static_cast<int>(blockIdx.x) / p.splits;  // b * Hkv + kvh
-  const int split = static_cast<int>(blockIdx.x) - bkv * p.splits;
-  const int b = bkv / p.Hkv, kvh = bkv - b * p.Hkv;
-  const int k_begin = split * p.keys_per_split;
-  const int k_end = min(p.Nk, k_begin + p.keys_per_split);
-  const int ntiles = k_end > k_begin ? (k_end - k_begin + KT - 1) / KT : 0;
-  const int R = p.R;
+  // this CTA's work units [u0, u0 + n): unit u = (KV head u / tiles, key tile u % tiles)
+  const int cta = static_cast<int>(blockIdx.x);
+  const long long u0 = static_cast<long long>(cta) * p.units / p.ctas;
+  const int n = static_cast<int>(static_cast<long long>(cta + 1) * p.units / p.ctas - u0);
 
   if (tid == 0) {
-    for (int s = 0; s < NSTAGE; ++s) mbar_init(base + C::OFF_BAR + 8 * s, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, NCW);
+    }
+    mbar_init(bar_gather, NCW);
+    mbar_init(bar_comb, NCW);
     *abort = 0;
     fence_barrier_init();
   }
   __syncthreads();
 
-  auto issue = [&](int t) {
-    const int s = t % NSTAGE;
-    const uint32_t bar = base + C::OFF_BAR + 8 * s;
-    mbar_arrive_expect_tx(bar, 2 * C::TILE);
-    for (int bx = 0; bx < D / 64; ++bx) {
-      tma_load_3d(base + C::OFF_K + s * C::TILE + bx * C::BOX, &tmK, bar, bx * 64, k_begin + t * KT, bkv);
-      tma_load_3d(base + C::OFF_V + s * C::TILE + bx * C::BOX, &tmV, bar, bx * 64, k_begin + t * KT, bkv);
+  if (warp == NCW) {
+    // ---- producer: one thread streams K and V tiles through the ring
+    if (lane != 0) return;
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    int issued = 0;
+    for (int i = 0; i < n; ++i) {
+      const int s = i % NST;
+      if (i >= NST && !mbar_wait(bar_empty + 8 * s, ((i / NST) - 1) & 1, abort, p.status, SITE_BWD + 21)) break;
+      const long long u = u0 + i;
+      const int bkv = static_cast<int>(u / p.tiles);
+      const int t = static_cast<int>(u - static_cast<long long>(bkv) * p.tiles);
+      const uint32_t dst = base + s * C::STAGE;
+      mbar_arrive_expect_tx(bar_full + 8 * s, 2 * C::TILE);
+      for (int bx = 0; bx < D / 64; ++bx) {
+        tma_load_3d(dst + bx * C::BOX, &tmK, bar_full + 8 * s, bx * 64, t * KT, bkv);
+        tma_load_3d(dst + C::TILE + bx * C::BOX, &tmV, bar_full + 8 * s, bx * 64, t * KT, bkv);
+      }
+      issued = i + 1;
     }
-  };
-  if (tid == 0)
-    for (int t = 0; t < ntiles && t < NSTAGE - 1; ++t) issue(t);
-
-  // Q fragments (A operand, rows = query rows of this KV head, k = d), kept in
-  // registers: row r = (head in group) * Nq + query index; rows >= R are 0.
-  uint32_t qa[D / 16][4];
-  {
-    auto qword = [&](int r, int c) -> uint32_t {  // bf16 pair (c, c + 1) of row r
-      if (r >= R) return 0u;
-      const int hq = kvh * p.group + r / p.Nq, qi = r % p.Nq;
-      return *reinterpret_cast<const uint32_t*>(p.q + ((static_cast<long long>(b) * p.Hq + hq) * p.Nq + qi) * D + c);
-    };
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      qa[ks][0] = qword(g4, 16 * ks + 2 * t4);
-      qa[ks][1] = qword(g4 + 8, 16 * ks + 2 * t4);
-      qa[ks][2] = qword(g4, 16 * ks + 8 + 2 * t4);
-      qa[ks][3] = qword(g4 + 8, 16 * ks + 8 + 2 * t4);
+    // Stay until the last copies have landed (they may outlive the consumers
+    // if those give up on a wait); each wait is bounded.
+    for (int i = issued > NST ? issued - NST : 0; i < issued; ++i) {
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(bar_full + 8 * (i % NST), (i / NST) & 1))
+        if (globaltimer() - t0 > 100000000ull) break;
     }
+    return;
   }
+
+  // ---- consumers: warp w owns keys 16w .. 16w + 15 of every tile and keeps
+  // its own running max, sum and O for them; the warps' results for a KV head
+  // are merged when the CTA's range of that head ends.
+  const int g4 = lane >> 2, t4 = lane & 3;  // mma fragment row group and column pair
+  const int mi = lane >> 3, ri = lane & 7;  // ldmatrix: matrix and row this lane addresses
+  const int R = p.R;
+  const int kw = 16 * warp;
   // query position in the sequence of fragment rows g4 and g4 + 8 (causal mask)
   const int qpos0 = (g4 % p.Nq) + p.Nk - p.Nq, qpos1 = ((g4 + 8) % p.Nq) + p.Nk - p.Nq;
 
-  // running max / sum of the two rows this warp owns in the softmax
-  float m_row[2] = {-INFINITY, -INFINITY}, l_row[2] = {0.f, 0.f};
-  // P V accumulators: rows g4, g4 + 8; columns of this warp's NB 8-column blocks
-  float acc[C::NB][4];
-#pragma unroll
-  for (int nb = 0; nb < C::NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-  int t_stop = ntiles;  // first tile not consumed (set on abort)
+  uint32_t qa[D / 16][4];  // Q fragments of the current KV head (A operand, k = d)
+  float m_r[2];            // running max of rows g4, g4 + 8 over this warp's keys (same across a quad)
+  float l_r[2];            // this thread's share of the running sums
+  float acc[D / 8][4];     // O rows g4, g4 + 8; columns 8 nb + 2 t4, + 1
 
-  for (int t = 0; t < ntiles; ++t) {
-    const int s = t % NSTAGE;
-    if (tid == 0 && t + NSTAGE - 1 < ntiles) issue(t + NSTAGE - 1);  // its stage was released at the end of t-1
-    const bool got = mbar_wait(base + C::OFF_BAR + 8 * s, (t / NSTAGE) & 1, abort, p.status, SITE_BWD + 20);
-    if (__syncthreads_or(!got)) {
-      t_stop = t;
+  int bkv = static_cast<int>(u0 / p.tiles);
+  int t = static_cast<int>(u0 - static_cast<long long>(bkv) * p.tiles);
+  int nseg = 0;  // head ranges merged so far (phase of the gather / combine barriers)
+
+  for (int i = 0; i < n; ++i) {
+    const int s = i % NST;
+    if (i == 0 || t == 0) {
+      // a new KV head: its query rows (row r = head in group * Nq + query; rows >= R are 0)
+      const int b = bkv / p.Hkv, kvh = bkv - b * p.Hkv;
+      auto qword = [&](int r, int c) -> uint32_t {  // bf16 pair (c, c + 1) of row r
+        if (r >= R) return 0u;
+        const int hq = kvh * p.group + r / p.Nq, qi = r % p.Nq;
+        return *reinterpret_cast<const uint32_t*>(p.q + ((static_cast<long long>(b) * p.Hq + hq) * p.Nq + qi) * D + c);
+      };
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        qa[ks][0] = qword(g4, 16 * ks + 2 * t4);
+        qa[ks][1] = qword(g4 + 8, 16 * ks + 2 * t4);
+        qa[ks][2] = qword(g4, 16 * ks + 8 + 2 * t4);
+        qa[ks][3] = qword(g4 + 8, 16 * ks + 8 + 2 * t4);
+      }
+      m_r[0] = m_r[1] = -INFINITY;
+      l_r[0] = l_r[1] = 0.f;
+#pragma unroll
+      for (int nb = 0; nb < D / 8; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
+    }
+    if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, (i / NST) & 1, abort, p.status, SITE_BWD + 22)))
       break;
-    }
-    const uint32_t kt = base + C::OFF_K + s * C::TILE;
-    const uint32_t vt = base + C::OFF_V + s * C::TILE;
-    const int kt0 = k_begin + t * KT;
-    // ---- S = Q K^T for keys 8w .. 8w + 7
-    {
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
-      const int mi = lane >> 3, ri = lane & 7;  // ldmatrix: matrix and row this lane addresses
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ks += 2) {
-        uint32_t b0, b1, b2, b3;  // (k-step ks: d 0-7, 8-15), (k-step ks + 1: d 0-7, 8-15)
-        ldsm_x4(kt + tile_off(8 * warp + ri, 16 * ks + 8 * mi), b0, b1, b2, b3);
-        mma16816(sc, qa[ks], b0, b1);
-        mma16816(sc, qa[ks + 1], b2, b3);
-      }
-      const int key0 = kt0 + 8 * warp + 2 * t4;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kg = key0 + (e & 1);
-        const int qpos = e < 2 ? qpos0 : qpos1;
-        const bool vis = kg < k_end && (!p.causal || kg <= qpos);
-        ssc[(g4 + 8 * (e >> 1)) * SS + 8 * warp + 2 * t4 + (e & 1)] = vis ? sc[e] * p.scale_log2 : -INFINITY;
-      }
-    }
-    __syncthreads();
-    // ---- softmax: warp w takes rows 2w and 2w + 1 (rows >= R get P = 0)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int r = 2 * warp + h;
-      float p0 = 0.f, p1 = 0.f;
-      if (r < R) {
-        const float s0 = ssc[r * SS + lane], s1 = ssc[r * SS + lane + 32];
-        float mx = fmaxf(s0, s1);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float m_new = fmaxf(m_row[h], mx);
-        const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        const float alpha = m_row[h] == -INFINITY ? 0.f : ex2(m_row[h] - m_use);
-        p0 = ex2(s0 - m_use);
-        p1 = ex2(s1 - m_use);
-        float sum = p0 + p1;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        l_row[h] = l_row[h] * alpha + sum;
-        m_row[h] = m_new;
-        if (lane == 0) salpha[r] = alpha;
-      } else if (lane == 0) {
-        salpha[r] = 0.f;
-      }
-      const uint32_t w01 = pack_bf16x2(p0, p1);
-      sp[r * PS + lane] = static_cast<uint16_t>(w01 & 0xFFFFu);
-      sp[r * PS + lane + 32] = static_cast<uint16_t>(w01 >> 16);
-    }
-    __syncthreads();
-    // ---- O += P V for this warp's columns
-    {
-      const float a0 = salpha[g4], a1 = salpha[g4 + 8];
-#pragma unroll
-      for (int nb = 0; nb < C::NB; ++nb) {
-        acc[nb][0] *= a0;
-        acc[nb][1] *= a0;
-        acc[nb][2] *= a1;
-        acc[nb][3] *= a1;
-      }
-      const int mi = lane >> 3, ri = lane & 7;
-      const uint32_t pbase = smem_u32(sp);
-#pragma unroll
-      for (int ks = 0; ks < KT / 16; ++ks) {
-        uint32_t pa[4];  // A: rows 0-7 / 8-15 x keys 16ks + 0-7 / 8-15
-        ldsm_x4(pbase + (((mi & 1) * 8 + ri) * PS + 16 * ks + (mi >> 1) * 8) * 2, pa[0], pa[1], pa[2], pa[3]);
-        const int col0 = C::NB * 8 * warp;
-        if (C::NB == 2) {
-          uint32_t b0, b1, b2, b3;  // (keys 0-7, 8-15) x (columns col0.., col0 + 8..)
-          ldsm_x4_t(vt + tile_off(16 * ks + (mi & 1) * 8 + ri, col0 + (mi >> 1) * 8), b0, b1, b2, b3);
-          mma16816(acc[0], pa, b0, b1);
-          mma16816(acc[C::NB - 1], pa, b2, b3);
-        } else {
-          uint32_t b0, b1;
-          ldsm_x2_t(vt + tile_off(16 * ks + (mi & 1) * 8 + ri, col0), b0, b1);
-          mma16816(acc[0], pa, b0, b1);
-        }
-      }
-    }
-    __syncthreads();  // this stage, the scores and P are free again
-  }
+    const uint32_t st = base + s * C::STAGE;  // K tile, then the V tile at + TILE
 
-  // partial results of this split, normalised within the split
-  if (t_stop == ntiles) {
+    // ---- S = Q K^T for this warp's keys (two 8-key blocks), base-2 scaled and masked
+    float sc[2][4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int r = 2 * warp + h;
-      if (r < R && lane == 0) {
-        salpha[r] = l_row[h] > 0.f ? 1.0f / l_row[h] : 0.f;
-        p.lse_part[(static_cast<long long>(bkv) * p.splits + split) * R + r] =
-            l_row[h] > 0.f ? (m_row[h] + __log2f(l_row[h])) * LN2 : -INFINITY;
-      }
+    for (int nb = 0; nb < 2; ++nb) sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t b0, b1, b2, b3;  // keys kw + 0-7: d lo, d hi; keys kw + 8-15: d lo, d hi
+      ldsm_x4(st + tile_off(kw + 8 * (mi >> 1) + ri, 16 * ks + 8 * (mi & 1)), b0, b1, b2, b3);
+      mma16816(sc[0], qa[ks], b0, b1);
+      mma16816(sc[1], qa[ks], b2, b3);
     }
-    __syncthreads();
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+    {
+      const int key0 = t * KT + kw + 2 * t4;
 #pragma unroll
-    for (int nb = 0; nb < C::NB; ++nb) {
-      const int col = C::NB * 8 * warp + 8 * nb + 2 * t4;
+      for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int r = g4 + 8 * hh;
-        if (r < R) {
-          const float inv = salpha[r];
-          float2 v2 = make_float2(acc[nb][2 * hh] * inv, acc[nb][2 * hh + 1] * inv);
-          *reinterpret_cast<float2*>(p.o_part + ((static_cast<long long>(bkv) * p.splits + split) * R + r) * D + col) =
-              v2;
+        for (int e = 0; e < 4; ++e) {
+          const int kg = key0 + 8 * nb + (e & 1);
+          const bool vis = kg < p.Nk && (!p.causal || kg <= (e < 2 ? qpos0 : qpos1));
+          sc[nb][e] = vis ? sc[nb][e] * p.scale_log2 : -INFINITY;
+          if (e < 2) mx0 = fmaxf(mx0, sc[nb][e]);
+          else mx1 = fmaxf(mx1, sc[nb][e]);
         }
+    }
+#pragma unroll
+    for (int off = 1; off <= 2; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    // ---- online softmax; O and the sums are rescaled only when a row's max grew
+    {
+      const float n0 = fmaxf(m_r[0], mx0), n1 = fmaxf(m_r[1], mx1);
+      if (__any_sync(0xffffffffu, n0 > m_r[0] || n1 > m_r[1])) {
+        const float a0 = m_r[0] == -INFINITY ? 0.f : ex2(m_r[0] - n0);
+        const float a1 = m_r[1] == -INFINITY ? 0.f : ex2(m_r[1] - n1);
+#pragma unroll
+        for (int nb = 0; nb < D / 8; ++nb) {
+          acc[nb][0] *= a0;
+          acc[nb][1] *= a0;
+          acc[nb][2] *= a1;
+          acc[nb][3] *= a1;
+        }
+        l_r[0] *= a0;
+        l_r[1] *= a1;
+        m_r[0] = n0;
+        m_r[1] = n1;
       }
     }
-  } else if (tid == 0) {
-    // let the copies still in flight (tiles t_stop .. t_stop + NSTAGE - 1) land
-    // before the CTA exits; each wait is bounded
-    for (int t = t_stop; t < ntiles && t < t_stop + NSTAGE; ++t) {
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(base + C::OFF_BAR + 8 * (t % NSTAGE), (t / NSTAGE) & 1))
-        if (globaltimer() - t0 > 100000000ull) break;
+    uint32_t pa[4];  // P as the A operand of P V: rows g4 / g4 + 8, keys 2 t4 (+8)
+    {
+      const float mu0 = m_r[0] == -INFINITY ? 0.f : m_r[0];
+      const float mu1 = m_r[1] == -INFINITY ? 0.f : m_r[1];
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb) {
+        const float p0 = ex2(sc[nb][0] - mu0), p1 = ex2(sc[nb][1] - mu0);
+        const float p2 = ex2(sc[nb][2] - mu1), p3 = ex2(sc[nb][3] - mu1);
+        l_r[0] += p0 + p1;
+        l_r[1] += p2 + p3;
+        pa[2 * nb] = pack_bf16x2(p0, p1);
+        pa[2 * nb + 1] = pack_bf16x2(p2, p3);
+      }
+    }
+    // ---- O += P V over this warp's 16 keys, 16 columns per ldmatrix
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+      uint32_t b0, b1, b2, b3;  // keys 0-7 / 8-15 of columns 16c + 0-7, then of 16c + 8-15
+      ldsm_x4_t(st + C::TILE + tile_off(kw + 8 * (mi & 1) + ri, 16 * c + 8 * (mi >> 1)), b0, b1, b2, b3);
+      mma16816(acc[2 * c], pa, b0, b1);
+      mma16816(acc[2 * c + 1], pa, b2, b3);
+    }
+
+    if (i == n - 1 || t == p.tiles - 1) {
+      // The CTA's range of this KV head ends. The warps' partial outputs go
+      // into this stage (every warp has read it), then each thread merges a
+      // share of the R x D output and writes the CTA's partial result to slot
+      // cta + bkv, rows normalised within the range.
+      float l0 = l_r[0], l1 = l_r[1];
+#pragma unroll
+      for (int off = 1; off <= 2; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_gather);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_gather, nseg & 1, abort, p.status, SITE_BWD + 23))) break;
+      float* const buf = reinterpret_cast<float*>(bp + s * C::STAGE);  // [NCW][MR][D]
+#pragma unroll
+      for (int nb = 0; nb < D / 8; ++nb) {
+        *reinterpret_cast<float2*>(buf + (warp * MR + g4) * D + 8 * nb + 2 * t4) = make_float2(acc[nb][0], acc[nb][1]);
+        *reinterpret_cast<float2*>(buf + (warp * MR + g4 + 8) * D + 8 * nb + 2 * t4) =
+            make_float2(acc[nb][2], acc[nb][3]);
+      }
+      if (t4 == 0) {
+        sml[(warp * MR + g4) * 2] = m_r[0];
+        sml[(warp * MR + g4) * 2 + 1] = l0;
+        sml[(warp * MR + g4 + 8) * 2] = m_r[1];
+        sml[(warp * MR + g4 + 8) * 2 + 1] = l1;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_comb);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_comb, nseg & 1, abort, p.status, SITE_BWD + 24))) break;
+      ++nseg;
+      const long long slot = static_cast<long long>(cta) + bkv;
+      for (int idx = tid; idx < R * D; idx += NCW * 32) {
+        const int r = idx / D, col = idx - r * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NCW; ++w) M = fmaxf(M, sml[(w * MR + r) * 2]);
+        float L = 0.f, o = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < NCW; ++w) {
+            const float mw = sml[(w * MR + r) * 2];
+            if (mw != -INFINITY) {
+              const float f = ex2(mw - M);
+              L = fmaf(f, sml[(w * MR + r) * 2 + 1], L);
+              o = fmaf(f, buf[(w * MR + r) * D + col], o);
+            }
+          }
+        }
+        p.o_part[(slot * R + r) * D + col] = L > 0.f ? o / L : 0.f;
+        if (col == 0) p.lse_part[slot * R + r] = L > 0.f ? (M + __log2f(L)) * LN2 : -INFINITY;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_empty + 8 * s);  // this warp is done with the stage
+    if (++t == p.tiles) {
+      t = 0;
+      ++bkv;
     }
   }
 }
 
-// One warp per output row (b, hq, query): merge the splits by log-sum-exp.
+// One warp per output row (b, hq, query): merge the partial results of its KV
+// head by log-sum-exp. The CTAs that touched head bkv are the owners of its
+// first and last units; owner(u) = ((u + 1) * ctas - 1) / units.
 template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(const DecParams p, int rows) {
   const int w = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
@@ -287,39 +344,59 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const DecParams p, 
   const int b = bh / p.Hq, hq = bh - b * p.Hq;
   const int bkv = b * p.Hkv + hq / p.group;
   const int r = (hq % p.group) * p.Nq + qi;
+  const long long first_unit = static_cast<long long>(bkv) * p.tiles;
+  const long long c_first = ((first_unit + 1) * p.ctas - 1) / p.units;
+  const long long c_last = ((first_unit + p.tiles) * p.ctas - 1) / p.units;
+  const int nparts = static_cast<int>(c_last - c_first + 1);
+  const long long slot0 = c_first + bkv;
+
   float mx = -INFINITY;
-  for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.lse_part[(static_cast<long long>(bkv) * p.splits + s) * p.R + r]);
+  for (int j = lane; j < nparts; j += 32) mx = fmaxf(mx, p.lse_part[(slot0 + j) * p.R + r]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   float wsum = 0.f;
   float o[D / 32];
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) o[e] = 0.f;
-  for (int s = 0; s < p.splits; ++s) {
-    const long long base_row = (static_cast<long long>(bkv) * p.splits + s) * p.R + r;
-    const float l = p.lse_part[base_row];
-    if (l == -INFINITY) continue;
-    const float wgt = __expf(l - mx);
-    wsum += wgt;
+  for (int j0 = 0; j0 < nparts; j0 += 32) {
+    // lane j holds the weight of partial j0 + j
+    float wl = 0.f;
+    if (j0 + lane < nparts) {
+      const float l = p.lse_part[(slot0 + j0 + lane) * p.R + r];
+      wl = l == -INFINITY ? 0.f : __expf(l - mx);
+    }
+    wsum += wl;
+    const int cnt = min(32, nparts - j0);
+#pragma unroll 4
+    for (int j = 0; j < cnt; ++j) {
+      const float wgt = __shfl_sync(0xffffffffu, wl, j);
+      const float* src = p.o_part + ((slot0 + j0 + j) * p.R + r) * D + lane;
 #pragma unroll
-    for (int e = 0; e < D / 32; ++e) o[e] = fmaf(wgt, p.o_part[base_row * D + lane + 32 * e], o[e]);
+      for (int e = 0; e < D / 32; ++e) o[e] = fmaf(wgt, src[32 * e], o[e]);
+    }
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
   const float inv = 1.0f / wsum;
   const long long orow = static_cast<long long>(bh) * p.Nq + qi;
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) {
-    const float v = o[e] * inv;
-    const uint32_t bits = __float_as_uint(v);
+    const uint32_t bits = __float_as_uint(o[e] * inv);
     p.o[orow * D + lane + 32 * e] = static_cast<uint16_t>((bits + 0x7FFFu + ((bits >> 16) & 1u)) >> 16);
   }
   if (lane == 0) p.lse[orow] = mx + __logf(wsum);
 }
 
 template <int D>
+cudaError_t set_smem() {
+  return cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DecCfg<D>::SMEM);
+}
+
+template <int D>
 cudaError_t launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecParams& p, int B, cudaStream_t stream) {
-  using C = DecCfg<D>;
-  auto k1 = decode_split_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaError_t e = set_smem<D>();
   if (e != cudaSuccess) return e;
-  k1<<<B * p.Hkv * p.splits, THREADS, C::SMEM, stream>>>(tmK, tmV, p);
+  decode_split_kernel<D><<<p.ctas, THREADS, DecCfg<D>::SMEM, stream>>>(tmK, tmV, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int rows = B * p.Hq * p.Nq;
@@ -327,11 +404,38 @@ cudaError_t launch(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecPara
   return cudaGetLastError();
 }
 
+template <int D>
+int resident() {
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (set_smem<D>() != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_split_kernel<D>, THREADS, DecCfg<D>::SMEM) !=
+      cudaSuccess)
+    return 0;
+  return sms * per_sm;
+}
+
 }  // namespace
 
 cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecParams& p, int B, int d,
                           cudaStream_t stream) {
   return d == 64 ? launch<64>(tmK, tmV, p, B, stream) : launch<128>(tmK, tmV, p, B, stream);
+}
+
+int decode_resident_ctas(int d) {
+  // per device and head dimension, queried once (a racing first query just
+  // stores the same value twice)
+  static std::atomic<int> cache[64][2];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return d == 64 ? resident<64>() : resident<128>();
+  std::atomic<int>& c = cache[dev][d == 64 ? 0 : 1];
+  int v = c.load(std::memory_order_relaxed);
+  if (v == 0) {
+    v = d == 64 ? resident<64>() : resident<128>();
+    c.store(v, std::memory_order_relaxed);
+  }
+  return v;
 }
 
 }  // namespace fa

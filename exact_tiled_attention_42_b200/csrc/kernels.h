@@ -86,8 +86,8 @@ struct DecParams {
   const uint16_t* q;  // bf16 [B*Hq, Nq, d]
   uint16_t* o;        // bf16 [B*Hq, Nq, d]
   float* lse;         // [B*Hq, Nq]
-  float* o_part;      // workspace [B*Hkv, splits, R, d] fp32, normalised within the split
-  float* lse_part;    // workspace [B*Hkv, splits, R], natural log (-inf: no key in the split)
+  float* o_part;      // workspace [ctas + B*Hkv, R, d] fp32, each normalised within its key range
+  float* lse_part;    // workspace [ctas + B*Hkv, R], natural log (-inf: no visible key in the range)
   int* status;
   int Hq;
   int Hkv;
@@ -95,16 +95,23 @@ struct DecParams {
   int Nq;
   int Nk;
   int R;              // group * Nq query rows per KV head
-  int splits;
-  int keys_per_split; // multiple of 64
+  int tiles;          // 64-key tiles per KV head: ceil(Nk / 64)
+  int ctas;           // CTAs of the split pass (<= units)
+  long long units;    // B * Hkv * tiles: the (KV head, key tile) work units
   int causal;
   float scale_log2;
 };
 
-// Decode-shaped forward: split pass over key chunks (one CTA per KV head and
-// split) then the LSE-weighted combine. tmK/tmV: bf16 [B*Hkv, Nk, d], 64 x 64
-// boxes, 128B swizzle.
+// Decode-shaped forward. Split pass: CTA c takes the contiguous work units
+// [c*units/ctas, (c+1)*units/ctas) in (KV head, key tile) order and writes one
+// partial result per KV head it touches, to slot c + (b*Hkv + kv head). Then
+// the log-sum-exp merge. tmK/tmV: bf16 [B*Hkv, Nk, d], 64 x 64 boxes, 128B
+// swizzle.
 cudaError_t launch_decode(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecParams& p, int B, int d,
                           cudaStream_t stream);
+
+// CTAs of the decode split pass that fit on the current device at once
+// (0 if the device cannot be queried).
+int decode_resident_ctas(int d);
 
 }  // namespace fa

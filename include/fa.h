@@ -147,11 +147,12 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
 
 /*
  * Bytes of device workspace fa_fwd_decode needs for these sizes and
- * num_splits (0 = automatic, as in fa_fwd_decode): per KV head, split and
- * query row, one float32 partial output row and one float32 log-sum-exp.
- * Returns 0 for invalid or unsupported sizes.
+ * num_ctas (0 = automatic, as in fa_fwd_decode): for each CTA of the split
+ * pass and each KV head, a float32 partial output row and a float32
+ * log-sum-exp per query row. Independent of the device. Returns 0 for invalid
+ * or unsupported sizes.
  */
-size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits);
+size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_ctas);
 
 /*
  * Forward for few query rows against a long key sequence (decoding with a
@@ -162,20 +163,24 @@ size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, i
  * "What tiling changes"); the pages do not discuss decoding. With causal
  * non-zero the queries are the last Nq positions of the sequence: query i
  * keeps keys j <= i + Nk - Nq (requires Nk >= Nq).
- * The key sequence is split into num_splits chunks processed by separate
- * CTAs (0 = choose automatically: enough CTAs to fill the GPU, at least 256
- * keys each); their partial outputs, written to the workspace, are merged by
- * log-sum-exp. Supported: d = 64 or 128, and (Hq / Hkv) * Nq <= 16 query rows
- * per KV head (FA_ERR_UNSUPPORTED otherwise). causal with Nk < Nq is
+ * Work split: the (KV head, 64-key tile) pairs are divided evenly among the
+ * CTAs of a split pass, each taking a contiguous run; a second kernel merges
+ * the partial results of each head by log-sum-exp. num_ctas = 0 runs as many
+ * CTAs as fit on the current device at once (at most 1024); a positive value
+ * asks for that many (capped at the number of pairs). The result does not
+ * depend on the split beyond floating-point rounding.
+ * Supported: d = 64 or 128, and (Hq / Hkv) * Nq <= 16 query rows per KV head
+ * (FA_ERR_UNSUPPORTED otherwise). causal with Nk < Nq or num_ctas < 0 is
  * FA_ERR_INVALID_ARG. `workspace` is device memory of at least
- * fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits) bytes,
- * 16-byte aligned (FA_ERR_WORKSPACE / FA_ERR_MISALIGNED otherwise); it is
- * overwritten. Two kernels run on `stream`: the split pass, then the merge.
+ * fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_ctas) bytes, 16-byte
+ * aligned (FA_ERR_WORKSPACE / FA_ERR_MISALIGNED otherwise); it is
+ * overwritten. Two kernels run on `stream`. If a kernel gives up on a bounded
+ * wait (FA_ERR_TIMEOUT from fa_last_device_status), o and lse are undefined.
  */
 fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                         void* workspace, size_t workspace_bytes,
                         int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
-                        int num_splits, cudaStream_t stream);
+                        int num_ctas, cudaStream_t stream);
 
 /* Human-readable name of a status code (static storage, never null). */
 const char* fa_status_string(fa_status s);

@@ -115,14 +115,19 @@ def test_workspace_sizes_are_linear_in_n(lib):
 def test_decode_rejects_bad_arguments(lib):
     ws = lib.fa_decode_workspace_size(2, 8, 2, 1, 4096, 128, 0)
     assert ws > 0
-    def dec(Hq=8, Hkv=2, Nq=1, Nk=4096, d=128, causal=1, ws_bytes=ws, wsp=P, q=P):
-        return lib.fa_fwd_decode(q, P, P, P, P, wsp, ws_bytes, 2, Hq, Hkv, Nq, Nk, d, causal, 0.08, 0, None)
+    def dec(Hq=8, Hkv=2, Nq=1, Nk=4096, d=128, causal=1, ws_bytes=ws, wsp=P, q=P, ctas=0):
+        return lib.fa_fwd_decode(q, P, P, P, P, wsp, ws_bytes, 2, Hq, Hkv, Nq, Nk, d, causal, 0.08, ctas, None)
     assert dec(q=None) == 1
     assert dec(Nq=8, Nk=4) == 1               # causal with more queries than keys
     assert dec(Hq=8, Hkv=1, Nq=4) == 2        # 32 query rows per KV head
     assert dec(d=96) == 2
     assert dec(wsp=None) == 4
     assert dec(ws_bytes=ws - 1) == 4
+    assert dec(ctas=-1) == 1
+    # an explicit CTA count needs room for its partials; the automatic one is
+    # sized for at most 1024 CTAs, whatever the device
+    assert lib.fa_decode_workspace_size(2, 8, 2, 1, 4096, 128, 7) < ws
+    assert lib.fa_decode_workspace_size(2, 8, 2, 1, 4096, 128, 4096) == ws
     assert lib.fa_decode_workspace_size(2, 8, 1, 4, 4096, 128, 0) == 0
     # the workspace holds partial rows per split, not an Nq x Nk matrix
     assert lib.fa_decode_workspace_size(16, 32, 8, 1, 131072, 128, 0) < 64 * 2 ** 20

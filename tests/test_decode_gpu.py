@@ -23,9 +23,9 @@ def inputs(B, Hq, Hkv, Nq, Nk, d, seed):
     return dev, host
 
 
-def run(dev, causal, splits=0, scale=None):
+def run(dev, causal, ctas=0, scale=None):
     import exact_tiled_attention_42_b200 as fa
-    o, lse = fa.fa_fwd_decode(dev["q"], dev["k"], dev["v"], causal=causal, num_splits=splits, scale=scale)
+    o, lse = fa.fa_fwd_decode(dev["q"], dev["k"], dev["v"], causal=causal, num_ctas=ctas, scale=scale)
     torch.cuda.synchronize()
     assert fa.fa_last_device_status() == 0
     return to_f64(o), lse.cpu().numpy().astype(np.float64)
@@ -57,10 +57,13 @@ def test_several_query_rows(Hq, Hkv, Nq, Nk, causal):
     check(o, lse, o_ref, lse_ref)
 
 
-@pytest.mark.parametrize("splits", [1, 2, 3, 7, 64])
-def test_split_count_does_not_change_the_result(splits):
+@pytest.mark.parametrize("ctas", [1, 2, 3, 7, 64, 95, 10000])
+def test_cta_count_does_not_change_the_result(ctas):
+    """2 x 2 KV heads x 47 key tiles shared by 1 .. 94 CTAs (10000 is capped
+    at one tile per CTA): ranges that end mid-head, cover a whole head, or
+    span a head boundary."""
     dev, host = inputs(2, 8, 2, 2, 3000, 128, seed=501)
-    o, lse = run(dev, True, splits)
+    o, lse = run(dev, True, ctas)
     o_ref, lse_ref = oracle.attention_forward(host["q"], host["k"], host["v"], True, 128 ** -0.5)
     check(o, lse, o_ref, lse_ref)
 
@@ -85,3 +88,13 @@ def test_decode_workload_sampled():
         o_ref, lse_ref = oracle.attention_forward(host["q"][b:b + 1, hs], host["k"][b:b + 1, kv:kv + 1],
                                                   host["v"][b:b + 1, kv:kv + 1], True, w.scale)
         check(o[b:b + 1, hs], lse[b:b + 1, hs], o_ref, lse_ref)
+
+
+def test_split_that_some_rows_cannot_see():
+    """Nk = 129 as three 64-key tiles on three CTAs: with the causal mask
+    aligned to the sequence end, query rows 0..14 see no key of the last tile
+    (its partial log-sum-exp is -inf and must drop out of the merge)."""
+    dev, host = inputs(1, 1, 1, 16, 129, 128, seed=503)
+    o, lse = run(dev, True, 3)
+    o_ref, lse_ref = oracle.attention_forward(host["q"], host["k"], host["v"], True, 128 ** -0.5)
+    check(o, lse, o_ref, lse_ref)
