@@ -61,11 +61,6 @@ struct DecCfg {
   static_assert(NCW * MR * D * 4 == STAGE, "a stage holds the warps' partial outputs");
 };
 
-// Byte offset of element (row, col) in a tile of 64-row, 128B-swizzled boxes.
-__device__ __forceinline__ uint32_t tile_off(int row, int col) {
-  return (col >> 6) * (KT * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2;
-}
-
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
@@ -75,9 +70,6 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
 }
 // D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -129,12 +121,14 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     int issued = 0;
+    int bkv = static_cast<int>(u0 / p.tiles);
+    int t = static_cast<int>(u0 - static_cast<long long>(bkv) * p.tiles);
     for (int i = 0; i < n; ++i) {
       const int s = i % NST;
-      if (i >= NST && !mbar_wait(bar_empty + 8 * s, ((i / NST) - 1) & 1, abort, p.status, SITE_BWD + 21)) break;
-      const long long u = u0 + i;
-      const int bkv = static_cast<int>(u / p.tiles);
-      const int t = static_cast<int>(u - static_cast<long long>(bkv) * p.tiles);
+      // the producer waits most of the time: sleep rather than spin, so the
+      // consumer warp that shares its scheduler keeps the issue slots
+      if (i >= NST && !mbar_wait_sleep(bar_empty + 8 * s, ((i / NST) - 1) & 1, abort, p.status, SITE_BWD + 21))
+        break;
       const uint32_t dst = base + s * C::STAGE;
       mbar_arrive_expect_tx(bar_full + 8 * s, 2 * C::TILE);
       for (int bx = 0; bx < D / 64; ++bx) {
@@ -142,6 +136,10 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
         tma_load_3d(dst + C::TILE + bx * C::BOX, &tmV, bar_full + 8 * s, bx * 64, t * KT, bkv);
       }
       issued = i + 1;
+      if (++t == p.tiles) {
+        t = 0;
+        ++bkv;
+      }
     }
     // Stay until the last copies have landed (they may outlive the consumers
     // if those give up on a wait); each wait is bounded.
@@ -160,8 +158,24 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
   const int mi = lane >> 3, ri = lane & 7;  // ldmatrix: matrix and row this lane addresses
   const int R = p.R;
   const int kw = 16 * warp;
-  // query position in the sequence of fragment rows g4 and g4 + 8 (causal mask)
-  const int qpos0 = (g4 % p.Nq) + p.Nk - p.Nq, qpos1 = ((g4 + 8) % p.Nq) + p.Nk - p.Nq;
+  // Keys visible to fragment rows g4 and g4 + 8 are those below lim0 / lim1:
+  // Nk, or with the causal mask (query index r % Nq at sequence position
+  // r % Nq + Nk - Nq) that position + 1. Computed once, without a division.
+  int lim0 = p.Nk, lim1 = p.Nk;
+  if (p.causal) {
+    int q0 = g4, q1 = g4 + 8;
+    while (q0 >= p.Nq) q0 -= p.Nq;
+    while (q1 >= p.Nq) q1 -= p.Nq;
+    lim0 = q0 + p.Nk - p.Nq + 1;
+    lim1 = q1 + p.Nk - p.Nq + 1;
+  }
+  // Per-lane byte offsets of the ldmatrix rows in a 128B-swizzled 64-row box:
+  // the 16-byte chunk index is XOR-ed with the row's low three bits, so the
+  // k-step's chunk is applied below with one XOR. K: matrix mi holds keys
+  // kw + 8 (mi >> 1) + ri at d chunk (mi & 1); V: keys kw + 8 (mi & 1) + ri at
+  // column chunk (mi >> 1).
+  const uint32_t lane_k = (kw + 8 * (mi >> 1) + ri) * 128 + (((ri ^ (mi & 1)) & 7) << 4);
+  const uint32_t lane_v = (kw + 8 * (mi & 1) + ri) * 128 + (((ri ^ (mi >> 1)) & 7) << 4);
 
   uint32_t qa[D / 16][4];  // Q fragments of the current KV head (A operand, k = d)
   float m_r[2];            // running max of rows g4, g4 + 8 over this warp's keys (same across a quad)
@@ -175,12 +189,13 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
   for (int i = 0; i < n; ++i) {
     const int s = i % NST;
     if (i == 0 || t == 0) {
-      // a new KV head: its query rows (row r = head in group * Nq + query; rows >= R are 0)
+      // a new KV head: its query rows. Row r = (head in group) * Nq + query
+      // index, so the group's rows are consecutive in q from its first head's
+      // first query (b * Hq + kvh * group) * Nq; rows >= R are 0.
       const int b = bkv / p.Hkv, kvh = bkv - b * p.Hkv;
+      const uint16_t* const qg = p.q + ((static_cast<long long>(b) * p.Hq + kvh * p.group) * p.Nq) * D;
       auto qword = [&](int r, int c) -> uint32_t {  // bf16 pair (c, c + 1) of row r
-        if (r >= R) return 0u;
-        const int hq = kvh * p.group + r / p.Nq, qi = r % p.Nq;
-        return *reinterpret_cast<const uint32_t*>(p.q + ((static_cast<long long>(b) * p.Hq + hq) * p.Nq + qi) * D + c);
+        return r < R ? *reinterpret_cast<const uint32_t*>(qg + r * D + c) : 0u;
       };
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
@@ -194,7 +209,7 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
 #pragma unroll
       for (int nb = 0; nb < D / 8; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
     }
-    if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, (i / NST) & 1, abort, p.status, SITE_BWD + 22)))
+    if (!__all_sync(0xffffffffu, mbar_wait_sleep(bar_full + 8 * s, (i / NST) & 1, abort, p.status, SITE_BWD + 22)))
       break;
     const uint32_t st = base + s * C::STAGE;  // K tile, then the V tile at + TILE
 
@@ -205,7 +220,7 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       uint32_t b0, b1, b2, b3;  // keys kw + 0-7: d lo, d hi; keys kw + 8-15: d lo, d hi
-      ldsm_x4(st + tile_off(kw + 8 * (mi >> 1) + ri, 16 * ks + 8 * (mi & 1)), b0, b1, b2, b3);
+      ldsm_x4(st + (ks >> 2) * C::BOX + (lane_k ^ ((ks & 3) << 5)), b0, b1, b2, b3);
       mma16816(sc[0], qa[ks], b0, b1);
       mma16816(sc[1], qa[ks], b2, b3);
     }
@@ -216,8 +231,7 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
       for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int kg = key0 + 8 * nb + (e & 1);
-          const bool vis = kg < p.Nk && (!p.causal || kg <= (e < 2 ? qpos0 : qpos1));
+          const bool vis = key0 + 8 * nb + (e & 1) < (e < 2 ? lim0 : lim1);
           sc[nb][e] = vis ? sc[nb][e] * p.scale_log2 : -INFINITY;
           if (e < 2) mx0 = fmaxf(mx0, sc[nb][e]);
           else mx1 = fmaxf(mx1, sc[nb][e]);
@@ -265,7 +279,7 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
 #pragma unroll
     for (int c = 0; c < D / 16; ++c) {
       uint32_t b0, b1, b2, b3;  // keys 0-7 / 8-15 of columns 16c + 0-7, then of 16c + 8-15
-      ldsm_x4_t(st + C::TILE + tile_off(kw + 8 * (mi & 1) + ri, 16 * c + 8 * (mi >> 1)), b0, b1, b2, b3);
+      ldsm_x4_t(st + C::TILE + (c >> 2) * C::BOX + (lane_v ^ ((c & 3) << 5)), b0, b1, b2, b3);
       mma16816(acc[2 * c], pa, b0, b1);
       mma16816(acc[2 * c + 1], pa, b2, b3);
     }
@@ -283,7 +297,7 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_gather);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_gather, nseg & 1, abort, p.status, SITE_BWD + 23))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait_sleep(bar_gather, nseg & 1, abort, p.status, SITE_BWD + 23))) break;
       float* const buf = reinterpret_cast<float*>(bp + s * C::STAGE);  // [NCW][MR][D]
 #pragma unroll
       for (int nb = 0; nb < D / 8; ++nb) {
@@ -299,7 +313,7 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_comb);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_comb, nseg & 1, abort, p.status, SITE_BWD + 24))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait_sleep(bar_comb, nseg & 1, abort, p.status, SITE_BWD + 24))) break;
       ++nseg;
       const long long slot = static_cast<long long>(cta) + bkv;
       for (int idx = tid; idx < R * D; idx += NCW * 32) {
