@@ -148,6 +148,19 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
 }
 
 // ------------------------------------------------------------------ main kernel
+// (query head in the GQA group, query tile) of successive loop iterations:
+// the tile runs first..last-1, then the next head starts again at first.
+struct QWalk {
+  int head, tile, first, last;
+  __device__ QWalk(int first_tile, int num_tiles) : head(0), tile(first_tile), first(first_tile), last(num_tiles) {}
+  __device__ void next() {
+    if (++tile == last) {
+      tile = first;
+      ++head;
+    }
+  }
+};
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -216,8 +229,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  auto q_head = [&](int it) { return b * p.Hq + kvh * p.group + it / nq; };  // b * Hq + hq
-  auto q_tile = [&](int it) { return i0 + it % nq; };
+  // Iteration it visits query head (it / nq) of the group and query tile
+  // i0 + it % nq. Each role walks these in order with a QWalk (no division).
+  const int bhq0 = b * p.Hq + kvh * p.group;  // first query head of the group, as b * Hq + hq
   auto ds_smem = [&](int st) -> uint32_t {
     return C::DS_ALIAS ? base + C::OFF_DO + st * C::TILE_BYTES : base + C::OFF_DS;
   };
@@ -231,12 +245,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tma_load_3d(base + C::OFF_V + bx * C::BOX_BYTES, &tmV, bars.kv_full(), bx * 64, j * BT, bkv);
       }
       int issued = 0;
-      for (int it = 0; it < n_it; ++it) {
+      QWalk qw(i0, T);
+      for (int it = 0; it < n_it; ++it, qw.next()) {
         const int st = it & 1;
         const uint32_t ph = (it >> 1) & 1;
-        const int bhq = q_head(it);
-        const int i = q_tile(it);
-        if (!mbar_wait(bars.q_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 1)) break;
+        const int bhq = bhq0 + qw.head;
+        const int i = qw.tile;
+        if (!mbar_wait_sleep(bars.q_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 1)) break;
         mbar_arrive_expect_tx(bars.q_full(st), C::TILE_BYTES + 1024);
         for (int bx = 0; bx < C::BOXES; ++bx)
           tma_load_3d(base + C::OFF_Q + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, bars.q_full(st), bx * 64,
@@ -244,7 +259,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const long long voff = static_cast<long long>(bhq) * p.Npad + i * BT;
         bulk_load_1d(base + C::OFF_VEC + st * 1024, p.neg_lse2 + voff, 512, bars.q_full(st));
         bulk_load_1d(base + C::OFF_VEC + st * 1024 + 512, p.delta + voff, 512, bars.q_full(st));
-        if (!mbar_wait(bars.do_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 2)) {
+        if (!mbar_wait_sleep(bars.do_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 2)) {
           issued = 2 * it + 1;
           break;
         }
@@ -270,13 +285,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       constexpr uint32_t IDESC_TS = idesc_bf16(BT, D, false, true);
       constexpr uint32_t IDESC_DQ = idesc_bf16(BT, D, true, true);
       const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
-      bool ok = mbar_wait(bars.kv_full(), 0, abort, p.status, SITE_BWD + 3);
+      bool ok = mbar_wait_sleep(bars.kv_full(), 0, abort, p.status, SITE_BWD + 3);
       for (int it = 0; ok && it < n_it; ++it) {
         const int st = it & 1;
         const uint32_t ph = (it >> 1) & 1;
         const uint32_t sQ = base + C::OFF_Q + st * C::TILE_BYTES;
         const uint32_t sdO = base + C::OFF_DO + st * C::TILE_BYTES;
-        if (!mbar_wait(bars.q_full(st), ph, abort, p.status, SITE_BWD + 4)) break;
+        if (!mbar_wait_sleep(bars.q_full(st), ph, abort, p.status, SITE_BWD + 4)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K_j Q_i^T
@@ -285,8 +300,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                  IDESC_SS, kk > 0 ? 1u : 0u);
         }
         mma_commit(bars.s_full());
-        if (!mbar_wait(bars.do_full(st), ph, abort, p.status, SITE_BWD + 5)) break;
-        if (C::DQ_SHARES_DP && it > 0 && !mbar_wait(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
+        if (!mbar_wait_sleep(bars.do_full(st), ph, abort, p.status, SITE_BWD + 5)) break;
+        if (C::DQ_SHARES_DP && it > 0 && !mbar_wait_sleep(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
           break;
         tc_fence_after();
 #pragma unroll
@@ -296,23 +311,23 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                  IDESC_SS, kk > 0 ? 1u : 0u);
         }
         mma_commit(bars.dp_full());
-        if (!mbar_wait(bars.p_ready(), it & 1, abort, p.status, SITE_BWD + 7)) break;
+        if (!mbar_wait_sleep(bars.p_ready(), it & 1, abort, p.status, SITE_BWD + 7)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)  // dV += P^T dO_i
           mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, smem_desc_sw128(sdO + kk * 2048, C::BOX_BYTES, 1024),
                  IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bars.dv_done());
-        if (!mbar_wait(bars.dst_ready(), it & 1, abort, p.status, SITE_BWD + 8)) break;
+        if (!mbar_wait_sleep(bars.dst_ready(), it & 1, abort, p.status, SITE_BWD + 8)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)  // dK += dS^T Q_i
           mma_ts(tmem + C::COL_DK, tmem + C::COL_S + 64 + kk * 8, smem_desc_sw128(sQ + kk * 2048, C::BOX_BYTES, 1024),
                  IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bars.q_empty(st));
-        if (!mbar_wait(bars.dss_ready(), it & 1, abort, p.status, SITE_BWD + 16)) break;
+        if (!mbar_wait_sleep(bars.dss_ready(), it & 1, abort, p.status, SITE_BWD + 16)) break;
         if (!C::DQ_SHARES_DP && it > 0 &&
-            !mbar_wait(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
+            !mbar_wait_sleep(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
           break;
         tc_fence_after();
         const uint32_t sdS = ds_smem(st);
@@ -333,12 +348,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t tDP = tmem + lane_off + C::COL_DP;
     const float cl2 = p.scale_log2;
     bool ok = true;
-    for (int it = 0; ok && it < n_it; ++it) {
+    QWalk qw(i0, T);
+    for (int it = 0; ok && it < n_it; ++it, qw.next()) {
       const int st = it & 1;
       const uint32_t ph = (it >> 1) & 1;
-      const int i = q_tile(it);
-      ok = __all_sync(0xffffffffu, mbar_wait(bars.q_full(st), ph, abort, p.status, SITE_BWD + 9));
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.s_full(), it & 1, abort, p.status, SITE_BWD + 10));
+      const int i = qw.tile;
+      ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.q_full(st), ph, abort, p.status, SITE_BWD + 9));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.s_full(), it & 1, abort, p.status, SITE_BWD + 10));
       if (!ok) break;
       tc_fence_after();
       const float* vec_lse = reinterpret_cast<const float*>(base_ptr + C::OFF_VEC + st * 1024);
@@ -389,7 +405,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.p_ready());
 
-      ok = __all_sync(0xffffffffu, mbar_wait(bars.dp_full(), it & 1, abort, p.status, SITE_BWD + 11));
+      ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.dp_full(), it & 1, abort, p.status, SITE_BWD + 11));
       if (!ok) break;
       tc_fence_after();
       // dS = P (dP - D), 32 queries at a time with P^T read back from tensor
@@ -415,7 +431,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.dst_ready());
-      ok = __all_sync(0xffffffffu, mbar_wait(bars.dv_done(), it & 1, abort, p.status, SITE_BWD + 12));
+      ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.dv_done(), it & 1, abort, p.status, SITE_BWD + 12));
       if (!ok) break;
       const uint32_t sdS = ds_smem(st);
 #pragma unroll
@@ -433,7 +449,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (lane == 0) mbar_arrive(bars.dss_ready());
     }
     // ------------------------------------------------------------ dK, dV epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.dkdv_done(), 0, abort, p.status, SITE_BWD + 13));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.dkdv_done(), 0, abort, p.status, SITE_BWD + 13));
     if (ok) {
       tc_fence_after();
       for (int which = 0; which < 2; ++which) {
@@ -461,7 +477,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.epi());
-      if (r == 0 && mbar_wait(bars.epi(), 0, abort, p.status, SITE_BWD + 14)) {
+      if (r == 0 && mbar_wait_sleep(bars.epi(), 0, abort, p.status, SITE_BWD + 14)) {
         for (int bx = 0; bx < C::BOXES; ++bx) {
           tma_store_3d(&tmdK, base + C::OFF_Q + bx * C::BOX_BYTES, bx * 64, j * BT, bkv);
           tma_store_3d(&tmdV, base + C::OFF_Q + C::TILE_BYTES + bx * C::BOX_BYTES, bx * 64, j * BT, bkv);
@@ -477,8 +493,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t stg0 = base + C::OFF_STG + w * 2 * 2048;
     int cnt = 0;
     bool ok = true;
+    QWalk qw(i0, T);
     for (int it = 0; ok && it < n_it; ++it) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bars.dq_full(), it & 1, abort, p.status, SITE_BWD + 15));
+      const int bhq = bhq0 + qw.head;
+      const int row0 = qw.tile * BT + w * 32;
+      qw.next();
+      ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.dq_full(), it & 1, abort, p.status, SITE_BWD + 15));
       if (!ok) break;
       tc_fence_after();
       float acc[D];
@@ -493,8 +513,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.dq_free());
-      const int bhq = q_head(it);
-      const int row0 = q_tile(it) * BT + w * 32;
       if (row0 >= p.N) continue;  // every row of this warp is padding
 #pragma unroll
       for (int c16 = 0; c16 < D / 16; ++c16) {

@@ -168,12 +168,12 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       for (int j = 0; j < nkv; ++j) {
         const int s = j % C::NS;
         const uint32_t ph = (j / C::NS) & 1;
-        if (!mbar_wait(bars.k_empty(s), ph ^ 1, abort, p.status, SITE_K_EMPTY)) break;
+        if (!mbar_wait_sleep(bars.k_empty(s), ph ^ 1, abort, p.status, SITE_K_EMPTY)) break;
         mbar_arrive_expect_tx(bars.k_full(s), C::TILE_BYTES);
         const uint32_t sK = base + C::OFF_K + s * C::TILE_BYTES;
         for (int bx = 0; bx < C::BOXES; ++bx)
           tma_load_3d(sK + bx * C::BOX_BYTES, &tmK, bars.k_full(s), bx * 64, j * BN, kvh);
-        if (!mbar_wait(bars.v_empty(s), ph ^ 1, abort, p.status, SITE_V_EMPTY)) {
+        if (!mbar_wait_sleep(bars.v_empty(s), ph ^ 1, abort, p.status, SITE_V_EMPTY)) {
           issued = 2 * j + 1;
           break;
         }
@@ -221,8 +221,8 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                  (accumulate || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&
-                mbar_wait(bars.k_full(0), 0, abort, p.status, SITE_K_FULL);
+      bool ok = mbar_wait_sleep(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&
+                mbar_wait_sleep(bars.k_full(0), 0, abort, p.status, SITE_K_FULL);
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
@@ -236,13 +236,13 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       for (int j = 1; ok && j <= nkv; ++j) {
         const int vs = (j - 1) % C::NS;
         const int ks = j % C::NS;
-        if (!mbar_wait(bars.v_full(vs), ((j - 1) / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
-        if (j < nkv && !mbar_wait(bars.k_full(ks), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) break;
+        if (!mbar_wait_sleep(bars.v_full(vs), ((j - 1) / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
+        if (j < nkv && !mbar_wait_sleep(bars.k_full(ks), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) break;
         tc_fence_after();
         for (int x = 0; x < 2; ++x) {
           const int nx = x ? n1 : n0;
           if (j - 1 >= nx) continue;
-          if (!mbar_wait(bars.p_full(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
+          if (!mbar_wait_sleep(bars.p_full(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
             ok = false;
             break;
           }
@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     for (int j = 0; ok && j < n; ++j) {
       // Every lane polls; the outcome is made warp-uniform before the
       // .sync.aligned tensor-memory instructions that follow.
-      if (!__all_sync(0xffffffffu, mbar_wait(bars.s_full(x), j & 1, abort, p.status, SITE_S_FULL))) {
+      if (!__all_sync(0xffffffffu, mbar_wait_sleep(bars.s_full(x), j & 1, abort, p.status, SITE_S_FULL))) {
         ok = false;
         break;
       }
@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.p_full(x));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.o_done(x), 0, abort, p.status, SITE_O_DONE));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.o_done(x), 0, abort, p.status, SITE_O_DONE));
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.0f / l;
@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.epi(x));
-      if (row == 0 && mbar_wait(bars.epi(x), 0, abort, p.status, SITE_O_DONE)) {
+      if (row == 0 && mbar_wait_sleep(bars.epi(x), 0, abort, p.status, SITE_O_DONE)) {
         for (int bx = 0; bx < C::BOXES; ++bx) tma_store_3d(&tmO, stage + bx * C::BOX_BYTES, bx * 64, qt * BM, bh);
         bulk_commit();
         bulk_wait_read0();
