@@ -43,7 +43,19 @@ constexpr int BM = 128;  // query rows per tile (tcgen05 M)
 constexpr int BN = 128;  // keys per tile
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
-constexpr int FWD_THREADS = 320;
+// Three full warpgroups: softmax of query tile 0 (warps 0-3) and tile 1
+// (warps 4-7); warpgroup 2 holds the producer and MMA warps and two warps
+// with no role. After setup warpgroup 2 gives registers back (setmaxnreg)
+// so the softmax warps, which keep a 128-score row each, can grow past the
+// 168 a thread is launched with (three warps share each scheduler's
+// register file) without spilling. The split adds up to the launch
+// allocation exactly: 256 * 208 + 128 * 88 = 384 * 168; the host checks the
+// compiled register count against it before launching.
+constexpr int FWD_THREADS = 384;
+constexpr int REGS_SOFTMAX = 208;
+constexpr int REGS_OTHER = 88;
+constexpr int REGS_AT_LAUNCH = 168;
+static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER <= FWD_THREADS * REGS_AT_LAUNCH, "register split");
 constexpr float TAU = 8.0f;
 constexpr float LN2 = 0.69314718055994530942f;
 
@@ -153,114 +165,119 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == PRODUCER_WARP) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint32_t sQ = base + C::OFF_Q;
-      mbar_arrive_expect_tx(bars.q_full(), (has1 ? 2 : 1) * C::TILE_BYTES);
-      for (int bx = 0; bx < C::BOXES; ++bx)
-        tma_load_3d(sQ + bx * C::BOX_BYTES, &tmQ, bars.q_full(), bx * 64, qt0 * BM, bh);
-      if (has1)
+  if (warp >= 8) {
+    // warpgroup 2: producer, MMA issuer and two warps without a role
+    setmaxnreg_dec<REGS_OTHER>();
+    if (warp == PRODUCER_WARP) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        const uint32_t sQ = base + C::OFF_Q;
+        mbar_arrive_expect_tx(bars.q_full(), (has1 ? 2 : 1) * C::TILE_BYTES);
         for (int bx = 0; bx < C::BOXES; ++bx)
-          tma_load_3d(sQ + C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, bars.q_full(), bx * 64, qt1 * BM, bh);
-      int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % C::NS;
-        const uint32_t ph = (j / C::NS) & 1;
-        if (!mbar_wait_sleep(bars.k_empty(s), ph ^ 1, abort, p.status, SITE_K_EMPTY)) break;
-        mbar_arrive_expect_tx(bars.k_full(s), C::TILE_BYTES);
-        const uint32_t sK = base + C::OFF_K + s * C::TILE_BYTES;
-        for (int bx = 0; bx < C::BOXES; ++bx)
-          tma_load_3d(sK + bx * C::BOX_BYTES, &tmK, bars.k_full(s), bx * 64, j * BN, kvh);
-        if (!mbar_wait_sleep(bars.v_empty(s), ph ^ 1, abort, p.status, SITE_V_EMPTY)) {
-          issued = 2 * j + 1;
-          break;
-        }
-        mbar_arrive_expect_tx(bars.v_full(s), C::TILE_BYTES);
-        const uint32_t sV = base + C::OFF_V + s * C::TILE_BYTES;
-        for (int bx = 0; bx < C::BOXES; ++bx)
-          tma_load_3d(sV + bx * C::BOX_BYTES, &tmV, bars.v_full(s), bx * 64, j * BN, kvh);
-        issued = 2 * j + 2;
-      }
-      if (*abort) {
-        // Let every copy already issued land before the CTA can exit.
-        drain_wait(bars.q_full(), 0);
-        for (int t = (issued > 2 * C::NS ? issued - 2 * C::NS : 0); t < issued; ++t) {
-          const int j = t >> 1;
-          const uint32_t bar = (t & 1) ? bars.v_full(j % C::NS) : bars.k_full(j % C::NS);
-          drain_wait(bar, (j / C::NS) & 1);
-        }
-      }
-    }
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
-      constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, false, true);
-      const uint32_t sQ = base + C::OFF_Q;
-      auto issue_qk = [&](int x, int stage) {
-        const uint32_t dS = tmem + (x ? C::COL_S1 : C::COL_S0);
-        const uint32_t qa = sQ + x * C::TILE_BYTES;
-        const uint32_t kb = base + C::OFF_K + stage * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          mma_ss(dS, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), IDESC_QK,
-                 kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int x, int stage, bool accumulate) {
-        const uint32_t dO = tmem + (x ? C::COL_O1 : C::COL_O0);
-        const uint32_t aP = tmem + (x ? C::COL_S1 : C::COL_S0);
-        const uint32_t vb = base + C::OFF_V + stage * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // 16 keys = two 8-row groups of the MN-major V tile; 16 bf16 of P = 8 columns.
-          mma_ts(dO, aP + kk * 8, smem_desc_sw128(vb + kk * 16 * 128, C::BOX_BYTES, 1024), IDESC_PV,
-                 (accumulate || kk > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait_sleep(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&
-                mbar_wait_sleep(bars.k_full(0), 0, abort, p.status, SITE_K_FULL);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, 0);
-        mma_commit(bars.s_full(0));
-        if (n1 > 0) {
-          issue_qk(1, 0);
-          mma_commit(bars.s_full(1));
-        }
-        mma_commit(bars.k_empty(0));
-      }
-      for (int j = 1; ok && j <= nkv; ++j) {
-        const int vs = (j - 1) % C::NS;
-        const int ks = j % C::NS;
-        if (!mbar_wait_sleep(bars.v_full(vs), ((j - 1) / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
-        if (j < nkv && !mbar_wait_sleep(bars.k_full(ks), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) break;
-        tc_fence_after();
-        for (int x = 0; x < 2; ++x) {
-          const int nx = x ? n1 : n0;
-          if (j - 1 >= nx) continue;
-          if (!mbar_wait_sleep(bars.p_full(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
-            ok = false;
+          tma_load_3d(sQ + bx * C::BOX_BYTES, &tmQ, bars.q_full(), bx * 64, qt0 * BM, bh);
+        if (has1)
+          for (int bx = 0; bx < C::BOXES; ++bx)
+            tma_load_3d(sQ + C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, bars.q_full(), bx * 64, qt1 * BM, bh);
+        int issued = 0;
+        for (int j = 0; j < nkv; ++j) {
+          const int s = j % C::NS;
+          const uint32_t ph = (j / C::NS) & 1;
+          if (!mbar_wait_sleep(bars.k_empty(s), ph ^ 1, abort, p.status, SITE_K_EMPTY)) break;
+          mbar_arrive_expect_tx(bars.k_full(s), C::TILE_BYTES);
+          const uint32_t sK = base + C::OFF_K + s * C::TILE_BYTES;
+          for (int bx = 0; bx < C::BOXES; ++bx)
+            tma_load_3d(sK + bx * C::BOX_BYTES, &tmK, bars.k_full(s), bx * 64, j * BN, kvh);
+          if (!mbar_wait_sleep(bars.v_empty(s), ph ^ 1, abort, p.status, SITE_V_EMPTY)) {
+            issued = 2 * j + 1;
             break;
           }
-          tc_fence_after();
-          issue_pv(x, vs, j > 1);
-          if (j < nx) {
-            issue_qk(x, ks);
-            mma_commit(bars.s_full(x));
-          } else {
-            mma_commit(bars.o_done(x));
+          mbar_arrive_expect_tx(bars.v_full(s), C::TILE_BYTES);
+          const uint32_t sV = base + C::OFF_V + s * C::TILE_BYTES;
+          for (int bx = 0; bx < C::BOXES; ++bx)
+            tma_load_3d(sV + bx * C::BOX_BYTES, &tmV, bars.v_full(s), bx * 64, j * BN, kvh);
+          issued = 2 * j + 2;
+        }
+        if (*abort) {
+          // Let every copy already issued land before the CTA can exit.
+          drain_wait(bars.q_full(), 0);
+          for (int t = (issued > 2 * C::NS ? issued - 2 * C::NS : 0); t < issued; ++t) {
+            const int j = t >> 1;
+            const uint32_t bar = (t & 1) ? bars.v_full(j % C::NS) : bars.k_full(j % C::NS);
+            drain_wait(bar, (j / C::NS) & 1);
           }
         }
-        if (!ok) break;
-        if (j < nkv) mma_commit(bars.k_empty(ks));
-        mma_commit(bars.v_empty(vs));
+      }
+    } else if (warp == MMA_WARP) {
+      // ------------------------------------------------------------ MMA issue
+      if (lane == 0) {
+        constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false, false);
+        constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, false, true);
+        const uint32_t sQ = base + C::OFF_Q;
+        auto issue_qk = [&](int x, int stage) {
+          const uint32_t dS = tmem + (x ? C::COL_S1 : C::COL_S0);
+          const uint32_t qa = sQ + x * C::TILE_BYTES;
+          const uint32_t kb = base + C::OFF_K + stage * C::TILE_BYTES;
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+            mma_ss(dS, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), IDESC_QK,
+                   kk > 0 ? 1u : 0u);
+          }
+        };
+        auto issue_pv = [&](int x, int stage, bool accumulate) {
+          const uint32_t dO = tmem + (x ? C::COL_O1 : C::COL_O0);
+          const uint32_t aP = tmem + (x ? C::COL_S1 : C::COL_S0);
+          const uint32_t vb = base + C::OFF_V + stage * C::TILE_BYTES;
+  #pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // 16 keys = two 8-row groups of the MN-major V tile; 16 bf16 of P = 8 columns.
+            mma_ts(dO, aP + kk * 8, smem_desc_sw128(vb + kk * 16 * 128, C::BOX_BYTES, 1024), IDESC_PV,
+                   (accumulate || kk > 0) ? 1u : 0u);
+          }
+        };
+        bool ok = mbar_wait_sleep(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&
+                  mbar_wait_sleep(bars.k_full(0), 0, abort, p.status, SITE_K_FULL);
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0);
+          mma_commit(bars.s_full(0));
+          if (n1 > 0) {
+            issue_qk(1, 0);
+            mma_commit(bars.s_full(1));
+          }
+          mma_commit(bars.k_empty(0));
+        }
+        for (int j = 1; ok && j <= nkv; ++j) {
+          const int vs = (j - 1) % C::NS;
+          const int ks = j % C::NS;
+          if (!mbar_wait_sleep(bars.v_full(vs), ((j - 1) / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
+          if (j < nkv && !mbar_wait_sleep(bars.k_full(ks), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) break;
+          tc_fence_after();
+          for (int x = 0; x < 2; ++x) {
+            const int nx = x ? n1 : n0;
+            if (j - 1 >= nx) continue;
+            if (!mbar_wait_sleep(bars.p_full(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(x, vs, j > 1);
+            if (j < nx) {
+              issue_qk(x, ks);
+              mma_commit(bars.s_full(x));
+            } else {
+              mma_commit(bars.o_done(x));
+            }
+          }
+          if (!ok) break;
+          if (j < nkv) mma_commit(bars.k_empty(ks));
+          mma_commit(bars.v_empty(vs));
+        }
       }
     }
-  } else if (warp < 8) {
+  } else {
+    // warpgroups 0 and 1: softmax
+    setmaxnreg_inc<REGS_SOFTMAX>();
     // ------------------------------------------------------------ softmax
     const int x = warp >> 2;  // query tile of this warpgroup
     const int qt = x ? qt1 : qt0;
@@ -405,6 +422,16 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
                    const FwdParams& p, int BH, cudaStream_t stream) {
   using C = FwdCfg<D>;
   auto kern = fwd_bf16_kernel<D, CAUSAL>;
+  // The softmax warpgroups' setmaxnreg.inc waits until the CTA's register
+  // pool has room; make sure the compiled launch allocation covers the split.
+  static int regs = 0;
+  if (regs == 0) {
+    cudaFuncAttributes fa_attr;
+    cudaError_t e0 = cudaFuncGetAttributes(&fa_attr, kern);
+    if (e0 != cudaSuccess) return e0;
+    regs = fa_attr.numRegs;
+  }
+  if (256 * REGS_SOFTMAX + 128 * REGS_OTHER > FWD_THREADS * regs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(BH * p.num_pairs);
