@@ -26,7 +26,16 @@ constexpr int BN = 128;
 constexpr int D = 128;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
-constexpr int THREADS = 320;
+// Three full warpgroups: softmax of query tile 0 (warps 0-3) and tile 1
+// (warps 4-7); warpgroup 2 holds the producer and MMA warps and two warps
+// with no role. After setup warpgroup 2 lowers its registers (setmaxnreg)
+// so the softmax warps can hold their score row without spilling past the
+// 168 a thread is launched with: 256 * 208 + 128 * 88 = 384 * 168, checked
+// against the compiled register count on the host before launching.
+constexpr int THREADS = 384;
+constexpr int REGS_SOFTMAX = 208;
+constexpr int REGS_OTHER = 88;
+static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * 168, "register split");
 constexpr float LN2 = 0.69314718055994530942f;
 constexpr float P_LIFT = 256.f;
 
@@ -149,98 +158,104 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == PRODUCER_WARP) {
-    if (lane == 0) {
-      const uint32_t sQ = base + C::OFF_Q;
-      mbar_arrive_expect_tx(bars.q_full(), (has1 ? 2 : 1) * C::TILE_BYTES);
-      tma_load_3d(sQ, &tmQ, bars.q_full(), 0, qt0 * BM, bh);
-      if (has1) tma_load_3d(sQ + C::TILE_BYTES, &tmQ, bars.q_full(), 0, qt1 * BM, bh);
-      int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % C::NS;
-        const uint32_t ph = (j / C::NS) & 1;
-        if (!mbar_wait(bars.k_empty(s), ph ^ 1, abort, p.status, SITE_K_EMPTY)) break;
-        mbar_arrive_expect_tx(bars.k_full(s), C::TILE_BYTES);
-        tma_load_3d(base + C::OFF_K + s * C::TILE_BYTES, &tmK, bars.k_full(s), 0, j * BN, kvh);
-        if (!mbar_wait(bars.v_empty(s), ph ^ 1, abort, p.status, SITE_V_EMPTY)) {
-          issued = 2 * j + 1;
-          break;
-        }
-        mbar_arrive_expect_tx(bars.v_full(s), C::TILE_BYTES);
-        tma_load_3d(base + C::OFF_V + s * C::TILE_BYTES, &tmV, bars.v_full(s), 0, j * BN, kvh);
-        issued = 2 * j + 2;
-      }
-      if (*abort) {
-        drain_wait(bars.q_full(), 0);
-        for (int t = (issued > 2 * C::NS ? issued - 2 * C::NS : 0); t < issued; ++t) {
-          const int j = t >> 1;
-          drain_wait((t & 1) ? bars.v_full(j % C::NS) : bars.k_full(j % C::NS), (j / C::NS) & 1);
-        }
-      }
-    }
-  } else if (warp == MMA_WARP) {
-    if (lane == 0) {
-      constexpr uint32_t IDESC_QK = idesc_e4m3(BM, BN, false, false);
-      constexpr uint32_t IDESC_PV = idesc_e4m3(BM, D, false, true);
-      const uint32_t sQ = base + C::OFF_Q;
-      auto issue_qk = [&](int x, int stage) {
-        const uint32_t dS = tmem + (x ? C::COL_S1 : C::COL_S0);
-        const uint32_t qa = sQ + x * C::TILE_BYTES;
-        const uint32_t kb = base + C::OFF_K + stage * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)  // 32 e4m3 = 32 bytes of each 128-byte row
-          mma_ss_f8(dS, smem_desc_sw128(qa + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 32, 16, 1024), IDESC_QK,
-                    kk > 0 ? 1u : 0u);
-      };
-      auto issue_pv = [&](int x, int stage, bool accumulate) {
-        const uint32_t dO = tmem + (x ? C::COL_O1 : C::COL_O0);
-        const uint32_t aP = tmem + (x ? C::COL_S1 : C::COL_S0);
-        const uint32_t vb = base + C::OFF_V + stage * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BN / 32; ++kk)  // 32 keys = four 8-row groups; 32 e4m3 of P = 8 columns
-          mma_ts_f8(dO, aP + kk * 8, smem_desc_sw128(vb + kk * 4096, 16384, 1024), IDESC_PV,
-                    (accumulate || kk > 0) ? 1u : 0u);
-      };
-      bool ok = mbar_wait(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&
-                mbar_wait(bars.k_full(0), 0, abort, p.status, SITE_K_FULL);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, 0);
-        mma_commit(bars.s_full(0));
-        if (n1 > 0) {
-          issue_qk(1, 0);
-          mma_commit(bars.s_full(1));
-        }
-        mma_commit(bars.k_empty(0));
-      }
-      for (int j = 1; ok && j <= nkv; ++j) {
-        const int vs = (j - 1) % C::NS;
-        const int ks = j % C::NS;
-        if (!mbar_wait(bars.v_full(vs), ((j - 1) / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
-        if (j < nkv && !mbar_wait(bars.k_full(ks), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) break;
-        tc_fence_after();
-        for (int x = 0; x < 2; ++x) {
-          const int nx = x ? n1 : n0;
-          if (j - 1 >= nx) continue;
-          if (!mbar_wait(bars.p_full(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
-            ok = false;
+  if (warp >= 8) {
+    // warpgroup 2: producer, MMA issuer and two warps without a role
+    setmaxnreg_dec<REGS_OTHER>();
+    if (warp == PRODUCER_WARP) {
+      if (lane == 0) {
+        const uint32_t sQ = base + C::OFF_Q;
+        mbar_arrive_expect_tx(bars.q_full(), (has1 ? 2 : 1) * C::TILE_BYTES);
+        tma_load_3d(sQ, &tmQ, bars.q_full(), 0, qt0 * BM, bh);
+        if (has1) tma_load_3d(sQ + C::TILE_BYTES, &tmQ, bars.q_full(), 0, qt1 * BM, bh);
+        int issued = 0;
+        for (int j = 0; j < nkv; ++j) {
+          const int s = j % C::NS;
+          const uint32_t ph = (j / C::NS) & 1;
+          if (!mbar_wait_sleep(bars.k_empty(s), ph ^ 1, abort, p.status, SITE_K_EMPTY)) break;
+          mbar_arrive_expect_tx(bars.k_full(s), C::TILE_BYTES);
+          tma_load_3d(base + C::OFF_K + s * C::TILE_BYTES, &tmK, bars.k_full(s), 0, j * BN, kvh);
+          if (!mbar_wait_sleep(bars.v_empty(s), ph ^ 1, abort, p.status, SITE_V_EMPTY)) {
+            issued = 2 * j + 1;
             break;
           }
-          tc_fence_after();
-          issue_pv(x, vs, j > 1);
-          if (j < nx) {
-            issue_qk(x, ks);
-            mma_commit(bars.s_full(x));
-          } else {
-            mma_commit(bars.o_done(x));
+          mbar_arrive_expect_tx(bars.v_full(s), C::TILE_BYTES);
+          tma_load_3d(base + C::OFF_V + s * C::TILE_BYTES, &tmV, bars.v_full(s), 0, j * BN, kvh);
+          issued = 2 * j + 2;
+        }
+        if (*abort) {
+          drain_wait(bars.q_full(), 0);
+          for (int t = (issued > 2 * C::NS ? issued - 2 * C::NS : 0); t < issued; ++t) {
+            const int j = t >> 1;
+            drain_wait((t & 1) ? bars.v_full(j % C::NS) : bars.k_full(j % C::NS), (j / C::NS) & 1);
           }
         }
-        if (!ok) break;
-        if (j < nkv) mma_commit(bars.k_empty(ks));
-        mma_commit(bars.v_empty(vs));
+      }
+    } else if (warp == MMA_WARP) {
+      if (lane == 0) {
+        constexpr uint32_t IDESC_QK = idesc_e4m3(BM, BN, false, false);
+        constexpr uint32_t IDESC_PV = idesc_e4m3(BM, D, false, true);
+        const uint32_t sQ = base + C::OFF_Q;
+        auto issue_qk = [&](int x, int stage) {
+          const uint32_t dS = tmem + (x ? C::COL_S1 : C::COL_S0);
+          const uint32_t qa = sQ + x * C::TILE_BYTES;
+          const uint32_t kb = base + C::OFF_K + stage * C::TILE_BYTES;
+  #pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk)  // 32 e4m3 = 32 bytes of each 128-byte row
+            mma_ss_f8(dS, smem_desc_sw128(qa + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 32, 16, 1024), IDESC_QK,
+                      kk > 0 ? 1u : 0u);
+        };
+        auto issue_pv = [&](int x, int stage, bool accumulate) {
+          const uint32_t dO = tmem + (x ? C::COL_O1 : C::COL_O0);
+          const uint32_t aP = tmem + (x ? C::COL_S1 : C::COL_S0);
+          const uint32_t vb = base + C::OFF_V + stage * C::TILE_BYTES;
+  #pragma unroll
+          for (int kk = 0; kk < BN / 32; ++kk)  // 32 keys = four 8-row groups; 32 e4m3 of P = 8 columns
+            mma_ts_f8(dO, aP + kk * 8, smem_desc_sw128(vb + kk * 4096, 16384, 1024), IDESC_PV,
+                      (accumulate || kk > 0) ? 1u : 0u);
+        };
+        bool ok = mbar_wait_sleep(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&
+                  mbar_wait_sleep(bars.k_full(0), 0, abort, p.status, SITE_K_FULL);
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0);
+          mma_commit(bars.s_full(0));
+          if (n1 > 0) {
+            issue_qk(1, 0);
+            mma_commit(bars.s_full(1));
+          }
+          mma_commit(bars.k_empty(0));
+        }
+        for (int j = 1; ok && j <= nkv; ++j) {
+          const int vs = (j - 1) % C::NS;
+          const int ks = j % C::NS;
+          if (!mbar_wait_sleep(bars.v_full(vs), ((j - 1) / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
+          if (j < nkv && !mbar_wait_sleep(bars.k_full(ks), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) break;
+          tc_fence_after();
+          for (int x = 0; x < 2; ++x) {
+            const int nx = x ? n1 : n0;
+            if (j - 1 >= nx) continue;
+            if (!mbar_wait_sleep(bars.p_full(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(x, vs, j > 1);
+            if (j < nx) {
+              issue_qk(x, ks);
+              mma_commit(bars.s_full(x));
+            } else {
+              mma_commit(bars.o_done(x));
+            }
+          }
+          if (!ok) break;
+          if (j < nkv) mma_commit(bars.k_empty(ks));
+          mma_commit(bars.v_empty(vs));
+        }
       }
     }
-  } else if (warp < 8) {
+  } else {
+    // warpgroups 0 and 1: softmax
+    setmaxnreg_inc<REGS_SOFTMAX>();
     const int x = warp >> 2;
     const int qt = x ? qt1 : qt0;
     const int n = x ? n1 : n0;
@@ -398,6 +413,16 @@ template <bool CAUSAL>
 cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
                    const Fp8Params& p, int BH, cudaStream_t stream) {
   auto kern = fwd_fp8_kernel<CAUSAL>;
+  // The softmax warpgroups' setmaxnreg.inc waits until the CTA's register
+  // pool has room; make sure the compiled launch allocation covers the split.
+  static int regs = 0;
+  if (regs == 0) {
+    cudaFuncAttributes fa_attr;
+    cudaError_t e0 = cudaFuncGetAttributes(&fa_attr, kern);
+    if (e0 != cudaSuccess) return e0;
+    regs = fa_attr.numRegs;
+  }
+  if (256 * REGS_SOFTMAX + 128 * REGS_OTHER > THREADS * regs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(BH * p.num_pairs);
