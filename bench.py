@@ -9,6 +9,13 @@ FLOPs follow the workload statement: 4*B*Hq*N^2*d for the forward, halved for
 the causal mask, and 2.5x that for the backward. Inputs (3 x 64 MiB) are
 larger than the 126 MB L2, so no flush runs between steps.
 
+The JSON line also carries: `e2e`, the same step through the public API with
+every step's inputs copied from pinned host memory and all results read back
+(three streams, two buffer sets: neighbouring steps' copies overlap the
+kernels); `fp8`, the FP8 workload's pre-pass + forward in TFLOP/s; `decode`,
+one decode step (a query row per head against a 16K-key cache) in GB/s against
+the measured HBM copy bandwidth.
+
 Multi-GPU: every (batch, head) is an independent problem, so ranks run the
 same per-GPU workload with no collective on the data path (weak scaling); the
 value is all ranks' FLOPs over the slowest rank's device time.
