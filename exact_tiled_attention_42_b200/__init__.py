@@ -13,6 +13,8 @@ from .api import (  # noqa: F401
     fa_bwd,
     fa_bwd_noalloc,
     fa_fwd_fp8,
+    fa_fp8_quantize,
+    fa_fwd_fp8_quantized,
     fa_fwd_decode,
     fa_decode_workspace_size,
     fa_bwd_workspace_size,

@@ -162,6 +162,45 @@ def fa_fwd_fp8(q, k, v, causal: bool = False, scale: float | None = None, rotati
     return out, lse
 
 
+def fa_fp8_quantize(q, k, v, rotation_seed: int = 0, use_rotation: bool = True, workspace=None, stream=None):
+    """The FP8 pre-pass alone: rotated (optional) and 64-row block-quantised
+    e4m3 copies of q, k, v with their scales, in a workspace (uint8 tensor)
+    that fa_fwd_fp8_quantized reads."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    _check("q", q, torch.bfloat16, (B, Hq, N, d))
+    _check("k", k, torch.bfloat16, (B, Hkv, N, d))
+    _check("v", v, torch.bfloat16, (B, Hkv, N, d))
+    if workspace is None:
+        workspace = torch.empty(max(fa_fp8_workspace_size(B, Hq, Hkv, N, d), 16), dtype=torch.uint8, device=q.device)
+    st = _lib.load().fa_fp8_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                     int(rotation_seed) & 0xFFFFFFFFFFFFFFFF, int(bool(use_rotation)),
+                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                     B, Hq, Hkv, N, d, _stream(stream))
+    if st != FA_OK:
+        raise FAError("fa_fp8_quantize", st)
+    return workspace
+
+
+def fa_fwd_fp8_quantized(workspace, shape, causal: bool = False, scale: float | None = None,
+                         use_rotation: bool = True, out=None, lse=None, stream=None):
+    """The FP8 forward from a workspace filled by fa_fp8_quantize;
+    shape = (B, Hq, Hkv, N, d) of the quantised tensors."""
+    B, Hq, Hkv, N, d = (int(x) for x in shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dev = workspace.device
+    out = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=dev) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev) if lse is None else lse
+    _check("out", out, torch.bfloat16, (B, Hq, N, d))
+    _check("lse", lse, torch.float32, (B, Hq, N))
+    st = _lib.load().fa_fwd_fp8_quantized(workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                          out.data_ptr(), lse.data_ptr(), int(bool(use_rotation)),
+                                          B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    if st != FA_OK:
+        raise FAError("fa_fwd_fp8_quantized", st)
+    return out, lse
+
+
 def fa_decode_workspace_size(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, num_ctas: int = 0) -> int:
     return int(_lib.load().fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_ctas))
 

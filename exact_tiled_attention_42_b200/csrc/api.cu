@@ -296,14 +296,18 @@ size_t fa_fp8_workspace_size(int B, int Hq, int Hkv, int N, int d) {
   return up1024(q * N * d) + 2 * up1024(kv * N * d) + up1024(q * nb * 4) + 2 * up1024(kv * nb * 4);
 }
 
-fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, uint64_t rotation_seed,
-                     int use_rotation, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d,
-                     int causal, float scale, cudaStream_t stream) {
-  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// Validates the FP8 arguments shared by the three FP8 entry points and fills
+// the parameter block (workspace layout: e4m3 Q, K, V codes, then the fp32
+// block scales of Q, K, V, each region 1024-byte aligned).
+fa_status fp8_setup(fa::Fp8Params* p, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d,
+                    float scale, int use_rotation) {
   fa_status st = check_shape(B, Hq, Hkv, N, d, scale);
   if (st != FA_OK) return st;
   if (d != 128) return FA_ERR_UNSUPPORTED;  // the FP8 kernels are built for d = 128
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < fa_fp8_workspace_size(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
   const long long BH = static_cast<long long>(B) * Hq, BHkv = static_cast<long long>(B) * Hkv;
@@ -312,39 +316,93 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
   char* ws = static_cast<char*>(workspace);
   const size_t cq = up1024(static_cast<size_t>(BH) * N * d), ckv = up1024(static_cast<size_t>(BHkv) * N * d);
   const size_t sq = up1024(static_cast<size_t>(BH) * nb * 4), skv = up1024(static_cast<size_t>(BHkv) * nb * 4);
-  fa::Fp8Params p;
-  p.src[0] = static_cast<const uint16_t*>(q);
-  p.src[1] = static_cast<const uint16_t*>(k);
-  p.src[2] = static_cast<const uint16_t*>(v);
-  p.codes[0] = reinterpret_cast<uint8_t*>(ws);
-  p.codes[1] = reinterpret_cast<uint8_t*>(ws + cq);
-  p.codes[2] = reinterpret_cast<uint8_t*>(ws + cq + ckv);
-  p.scales[0] = reinterpret_cast<float*>(ws + cq + 2 * ckv);
-  p.scales[1] = reinterpret_cast<float*>(ws + cq + 2 * ckv + sq);
-  p.scales[2] = reinterpret_cast<float*>(ws + cq + 2 * ckv + sq + skv);
-  p.heads[0] = static_cast<int>(BH);
-  p.heads[1] = static_cast<int>(BHkv);
-  p.heads[2] = static_cast<int>(BHkv);
-  p.rotation_seed = rotation_seed;
-  p.rotate = use_rotation != 0;
-  p.lse = lse;
-  p.status = status_ptr();
-  p.N = N;
-  p.nblk = nb;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.group = Hq / Hkv;
-  p.num_qtiles = (N + 127) / 128;
-  p.num_pairs = (p.num_qtiles + 1) / 2;
-  p.score_log2 = scale * 1.4426950408889634f / (p.rotate ? static_cast<float>(d) : 1.0f);
-  if (!p.status) return FA_ERR_CUDA;
+  p->src[0] = p->src[1] = p->src[2] = nullptr;
+  p->codes[0] = reinterpret_cast<uint8_t*>(ws);
+  p->codes[1] = reinterpret_cast<uint8_t*>(ws + cq);
+  p->codes[2] = reinterpret_cast<uint8_t*>(ws + cq + ckv);
+  p->scales[0] = reinterpret_cast<float*>(ws + cq + 2 * ckv);
+  p->scales[1] = reinterpret_cast<float*>(ws + cq + 2 * ckv + sq);
+  p->scales[2] = reinterpret_cast<float*>(ws + cq + 2 * ckv + sq + skv);
+  p->heads[0] = static_cast<int>(BH);
+  p->heads[1] = static_cast<int>(BHkv);
+  p->heads[2] = static_cast<int>(BHkv);
+  p->rotation_seed = 0;
+  p->rotate = use_rotation != 0;
+  p->lse = nullptr;
+  p->N = N;
+  p->nblk = nb;
+  p->Hq = Hq;
+  p->Hkv = Hkv;
+  p->group = Hq / Hkv;
+  p->num_qtiles = (N + 127) / 128;
+  p->num_pairs = (p->num_qtiles + 1) / 2;
+  p->score_log2 = scale * 1.4426950408889634f / (p->rotate ? static_cast<float>(d) : 1.0f);
+  p->status = nullptr;  // set by the caller once every argument has been checked
+  return FA_OK;
+}
+
+fa_status fp8_forward(const fa::Fp8Params& p, void* o, int B, int Hq, int Hkv, int N, int d, int causal,
+                      cudaStream_t stream) {
+  const long long BH = static_cast<long long>(B) * Hq, BHkv = static_cast<long long>(B) * Hkv;
   CUtensorMap tmQ, tmK, tmV, tmO;
   if (!make_map_e4m3(&tmQ, p.codes[0], d, N, BH) || !make_map_e4m3(&tmK, p.codes[1], d, N, BHkv) ||
       !make_map_e4m3(&tmV, p.codes[2], d, N, BHkv) || !make_map_bf16(&tmO, o, d, N, BH, 128))
     return FA_ERR_CUDA;
-  cudaError_t e = fa::launch_fp8_quant(p, stream);
-  if (e == cudaSuccess) e = fa::launch_fwd_fp8(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), causal != 0, stream);
+  cudaError_t e = fa::launch_fwd_fp8(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), causal != 0, stream);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fp8_quantize(const void* q, const void* k, const void* v, uint64_t rotation_seed, int use_rotation,
+                          void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d,
+                          cudaStream_t stream) {
+  if (!q || !k || !v) return FA_ERR_INVALID_ARG;
+  fa::Fp8Params p;
+  fa_status st = fp8_setup(&p, workspace, workspace_bytes, B, Hq, Hkv, N, d, 1.0f, use_rotation);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return FA_ERR_MISALIGNED;
+  p.src[0] = static_cast<const uint16_t*>(q);
+  p.src[1] = static_cast<const uint16_t*>(k);
+  p.src[2] = static_cast<const uint16_t*>(v);
+  p.rotation_seed = rotation_seed;
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+  return fa::launch_fp8_quant(p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd_fp8_quantized(const void* workspace, size_t workspace_bytes, void* o, float* lse, int use_rotation,
+                               int B, int Hq, int Hkv, int N, int d, int causal, float scale, cudaStream_t stream) {
+  if (!o || !lse) return FA_ERR_INVALID_ARG;
+  fa::Fp8Params p;
+  fa_status st = fp8_setup(&p, const_cast<void*>(workspace), workspace_bytes, B, Hq, Hkv, N, d, scale, use_rotation);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  p.lse = lse;
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+  return fp8_forward(p, o, B, Hq, Hkv, N, d, causal, stream);
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, uint64_t rotation_seed,
+                     int use_rotation, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d,
+                     int causal, float scale, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  fa::Fp8Params p;
+  fa_status st = fp8_setup(&p, workspace, workspace_bytes, B, Hq, Hkv, N, d, scale, use_rotation);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  p.src[0] = static_cast<const uint16_t*>(q);
+  p.src[1] = static_cast<const uint16_t*>(k);
+  p.src[2] = static_cast<const uint16_t*>(v);
+  p.rotation_seed = rotation_seed;
+  p.lse = lse;
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+  if (fa::launch_fp8_quant(p, stream) != cudaSuccess) return FA_ERR_CUDA;
+  return fp8_forward(p, o, B, Hq, Hkv, N, d, causal, stream);
 }
 
 }  // extern "C"

@@ -146,6 +146,31 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
                      cudaStream_t stream);
 
 /*
+ * The two halves of fa_fwd_fp8, for callers that quantise once and run the
+ * forward several times (a fixed key/value set), or that time the FP8
+ * forward apart from its pre-pass. fa_fwd_fp8 is exactly fa_fp8_quantize
+ * followed by fa_fwd_fp8_quantized on the same stream.
+ *
+ * fa_fp8_quantize: rotates (when use_rotation is non-zero) and block-quantises
+ * q, k, v (bf16) into `workspace`, in the layout described at fa_fwd_fp8.
+ * Same size rules and errors as fa_fwd_fp8.
+ */
+fa_status fa_fp8_quantize(const void* q, const void* k, const void* v,
+                          uint64_t rotation_seed, int use_rotation,
+                          void* workspace, size_t workspace_bytes,
+                          int B, int Hq, int Hkv, int N, int d, cudaStream_t stream);
+
+/*
+ * fa_fwd_fp8_quantized: the FP8 forward from a workspace that
+ * fa_fp8_quantize filled for the same B, Hq, Hkv, N, d and use_rotation
+ * (the rotation's 1/d is folded into the softmax scale, so use_rotation must
+ * match); the workspace is only read. Writes O (bf16) and LSE (float32).
+ */
+fa_status fa_fwd_fp8_quantized(const void* workspace, size_t workspace_bytes, void* o, float* lse,
+                               int use_rotation, int B, int Hq, int Hkv, int N, int d, int causal,
+                               float scale, cudaStream_t stream);
+
+/*
  * Bytes of device workspace fa_fwd_decode needs for these sizes and
  * num_ctas (0 = automatic, as in fa_fwd_decode): for each CTA of the split
  * pass and each KV head, a float32 partial output row and a float32

@@ -92,6 +92,14 @@ def test_fp8_rejects_bad_arguments(lib):
     assert lib.fa_fwd_fp8(P, P, P, P, P, 1, 1, None, ws, 1, 2, 2, 128, 128, 0, 0.1, None) == 4
     assert lib.fa_fwd_fp8(P, P, P, P, P, 1, 1, P, ws - 1, 1, 2, 2, 128, 128, 0, 0.1, None) == 4
     assert lib.fa_fwd_fp8(P, P, None, P, P, 1, 1, P, ws, 1, 2, 2, 128, 128, 0, 0.1, None) == 1
+    # the two halves take the same checks
+    assert lib.fa_fp8_quantize(P, P, P, 1, 1, None, ws, 1, 2, 2, 128, 128, None) == 4
+    assert lib.fa_fp8_quantize(P, None, P, 1, 1, P, ws, 1, 2, 2, 128, 128, None) == 1
+    assert lib.fa_fp8_quantize(P, P, P, 1, 1, P, ws, 1, 2, 2, 128, 64, None) == 2      # d = 64 not built
+    assert lib.fa_fwd_fp8_quantized(P, ws - 1, P, P, 1, 1, 2, 2, 128, 128, 0, 0.1, None) == 4
+    assert lib.fa_fwd_fp8_quantized(P, ws, None, P, 1, 1, 2, 2, 128, 128, 0, 0.1, None) == 1
+    assert lib.fa_fwd_fp8_quantized(P, ws, P + 2, P, 1, 1, 2, 2, 128, 128, 0, 0.1, None) == 3
+    assert lib.fa_fwd_fp8_quantized(P, ws, P, P, 1, 1, 3, 2, 128, 128, 0, 0.1, None) == 1  # Hq % Hkv
 
 
 def test_workspace_sizes_are_linear_in_n(lib):

@@ -164,3 +164,27 @@ def test_full_fp8_workload_sampled_error_report():
         print(f"head {h}: RMSE fp8 kernel {rmse_ours:.3e}, naive per-tensor fp8 {rmse_naive:.3e}, "
               f"ratio {rmse_naive / rmse_ours:.2f}")
         assert rmse_ours < rmse_naive
+
+
+@pytest.mark.parametrize("rotate", [True, False])
+@pytest.mark.parametrize("causal", [False, True])
+def test_quantize_then_forward_equals_one_call(rotate, causal):
+    """fa_fp8_quantize followed by fa_fwd_fp8_quantized runs the same kernels
+    on the same data as fa_fwd_fp8: identical bits; and a second forward
+    from the same workspace gives them again (the workspace is only read)."""
+    import exact_tiled_attention_42_b200 as fa
+    dev, _ = make_inputs(1, 4, 2, 640, 128, seed=611)
+    o1, lse1, ws1 = run_fp8(dev, causal, 17, rotate)
+    ws = fa.fa_fp8_quantize(dev["q"], dev["k"], dev["v"], rotation_seed=17, use_rotation=rotate)
+    shape = (1, 4, 2, 640, 128)
+    for _ in range(2):
+        o2, lse2 = fa.fa_fwd_fp8_quantized(ws, shape, causal=causal, use_rotation=rotate)
+        torch.cuda.synchronize()
+        assert fa.fa_last_device_status() == 0
+        np.testing.assert_array_equal(to_f64(o2), o1)
+        np.testing.assert_array_equal(lse2.cpu().numpy().astype(np.float64), lse1)
+    # the documented regions (the padding between them is never written)
+    c1, s1 = split_workspace(ws1, *shape)
+    c2, s2 = split_workspace(ws.cpu().numpy(), *shape)
+    for a, b in zip(c1 + s1, c2 + s2):
+        np.testing.assert_array_equal(a, b)
