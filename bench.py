@@ -166,6 +166,20 @@ def _oracle_threads():
         return os.cpu_count()
 
 
+def _host_info(threads) -> dict:
+    """The host the oracle ran on: CPU model, logical CPUs, BLAS threads."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "logical_cpus": os.cpu_count(), "blas_threads": threads}
+
+
 def _oracle_inputs(w):
     bits = attention_inputs(1, 1, 1, w.N, w.d, w.seed, with_dout=True)
     return {n: bf16_bits_to_f32(a).astype(np.float64) for n, a in bits.items()}
@@ -239,7 +253,8 @@ def run_reference(args, rank, world):
                    "passes": list(passes), "l2": "inputs larger than L2 (no flush between steps)"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"per step: query rows {rows[0]}..{rows[1] - 1} of one (batch, head) problem, "
-                                   f"fp64 numpy oracle, {len(passes)} pass(es)"},
+                                   f"fp64 numpy oracle, {len(passes)} pass(es)",
+                         "host": _host_info(threads)},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -405,7 +420,8 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_cpu_baseline:
         v, el, heads, threads = cpu_oracle_sample(w, causal, passes, seconds_budget=args.cpu_seconds)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": f"{heads} whole (batch, head) problem(s) of the workload, fp64 numpy, {el:.1f} s"}
+               "sample": f"{heads} whole (batch, head) problem(s) of the workload, fp64 numpy, {el:.1f} s",
+               "host": _host_info(threads)}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
