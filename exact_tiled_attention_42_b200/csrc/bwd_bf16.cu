@@ -21,14 +21,22 @@
 //   dV  += P^T dO_i       (P^T from tensor memory, bf16)
 //   dK  += dS^T Q_i       (dS^T from tensor memory, bf16)
 //   dQ_i = dS K_j         (dS from shared memory, MN-major)
-// Roles: warps 0-3 turn S^T into P^T and dP^T into dS^T (thread = key row);
-// warps 4-7 drain dQ_i out of tensor memory and add it into the fp32
-// accumulator with TMA reduce-add (thread = query row); warp 8 loads with TMA;
-// one thread of warp 9 issues every MMA. P^T and dS^T (bf16) are written over
-// the S^T columns; for d = 128 the dQ accumulator reuses the dP^T columns and
-// dS reuses the shared-memory slot of dO_i once dV has read it. dK is issued
-// as soon as dS^T is in tensor memory, before dS has reached shared memory
-// (which waits for dV), and dQ once it has.
+// Roles, 512 threads in four warpgroups: warpgroups 0 and 1 turn S^T into P^T
+// and dP^T into dS^T (thread = key row; query columns [0,64) and [64,128), so
+// two warps per scheduler share the exponentials); warpgroup 2 drains dQ_i out
+// of tensor memory and adds it into the fp32 accumulator with TMA reduce-add
+// (thread = query row), apart from the compute warps so that its reduce waits
+// never hold up the next P^T; in warpgroup 3, warp 12 loads with TMA and one
+// thread of warp 13 issues every MMA. A thread is launched with 128 registers
+// (four warps share each scheduler's register file); after setup warpgroup 3
+// lowers itself to 88 (setmaxnreg), the compute warpgroups rise to 136 and
+// the drain to 152 -- 256 * 136 + 128 * 152 + 128 * 88 = 512 * 128, checked
+// against the compiled register count on the host before launching.
+// Each compute warpgroup writes its P^T (bf16) over the first 32 of its 64
+// S^T columns and its dS^T over the next 32; for d = 128 the dQ accumulator
+// reuses the dP^T columns and dS reuses the shared-memory slot of dO_i once dV
+// has read it. dK is issued as soon as dS^T is in tensor memory, before dS has
+// reached shared memory (which waits for dV), and dQ once it has.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -36,9 +44,13 @@ namespace fa {
 namespace {
 
 constexpr int BT = 128;  // keys per CTA tile; queries per step
-constexpr int PRODUCER_WARP = 8;
-constexpr int MMA_WARP = 9;
-constexpr int BWD_THREADS = 320;
+constexpr int PRODUCER_WARP = 12;
+constexpr int MMA_WARP = 13;
+constexpr int BWD_THREADS = 512;
+constexpr int REGS_COMPUTE = 136;
+constexpr int REGS_DRAIN = 152;
+constexpr int REGS_OTHER = 88;
+static_assert(256 * REGS_COMPUTE + 128 * REGS_DRAIN + 128 * REGS_OTHER <= BWD_THREADS * 128, "register split");
 constexpr float LOG2E = 1.4426950408889634f;
 
 template <int D>
@@ -58,7 +70,7 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_VEC + 2048;
   static constexpr int NUM_BARS = 20;
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
-  static constexpr uint32_t COL_S = 0;    // S^T; then P^T bf16 in [0,64) and dS^T bf16 in [64,128)
+  static constexpr uint32_t COL_S = 0;    // S^T; then per 64 queries: P^T bf16 in +[0,32), dS^T in +[32,64)
   static constexpr uint32_t COL_DP = 128;
   static constexpr uint32_t COL_DV = 256;
   static constexpr uint32_t COL_DK = 256 + D;
@@ -201,9 +213,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
     mbar_init(bars.s_full(), 1);
     mbar_init(bars.dp_full(), 1);
-    mbar_init(bars.p_ready(), 4);
-    mbar_init(bars.dst_ready(), 4);
-    mbar_init(bars.dss_ready(), 4);
+    mbar_init(bars.p_ready(), 8);  // one arrive per compute warp (two warpgroups)
+    mbar_init(bars.dst_ready(), 8);
+    mbar_init(bars.dss_ready(), 8);
     mbar_init(bars.dv_done(), 1);
     mbar_init(bars.dq_full(), 1);
     mbar_init(bars.dq_free(), 4);
@@ -236,116 +248,126 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     return C::DS_ALIAS ? base + C::OFF_DO + st * C::TILE_BYTES : base + C::OFF_DS;
   };
 
-  if (warp == PRODUCER_WARP) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bars.kv_full(), 2 * C::TILE_BYTES);
-      for (int bx = 0; bx < C::BOXES; ++bx) {
-        tma_load_3d(base + C::OFF_K + bx * C::BOX_BYTES, &tmK, bars.kv_full(), bx * 64, j * BT, bkv);
-        tma_load_3d(base + C::OFF_V + bx * C::BOX_BYTES, &tmV, bars.kv_full(), bx * 64, j * BT, bkv);
-      }
-      int issued = 0;
-      QWalk qw(i0, T);
-      for (int it = 0; it < n_it; ++it, qw.next()) {
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        const int bhq = bhq0 + qw.head;
-        const int i = qw.tile;
-        if (!mbar_wait_sleep(bars.q_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 1)) break;
-        mbar_arrive_expect_tx(bars.q_full(st), C::TILE_BYTES + 1024);
-        for (int bx = 0; bx < C::BOXES; ++bx)
-          tma_load_3d(base + C::OFF_Q + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, bars.q_full(st), bx * 64,
-                      i * BT, bhq);
-        const long long voff = static_cast<long long>(bhq) * p.Npad + i * BT;
-        bulk_load_1d(base + C::OFF_VEC + st * 1024, p.neg_lse2 + voff, 512, bars.q_full(st));
-        bulk_load_1d(base + C::OFF_VEC + st * 1024 + 512, p.delta + voff, 512, bars.q_full(st));
-        if (!mbar_wait_sleep(bars.do_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 2)) {
-          issued = 2 * it + 1;
-          break;
+  if (warp >= 12) {
+    // warpgroup 3: producer, MMA issuer and two warps without a role
+    setmaxnreg_dec<REGS_OTHER>();
+    if (warp == PRODUCER_WARP) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bars.kv_full(), 2 * C::TILE_BYTES);
+        for (int bx = 0; bx < C::BOXES; ++bx) {
+          tma_load_3d(base + C::OFF_K + bx * C::BOX_BYTES, &tmK, bars.kv_full(), bx * 64, j * BT, bkv);
+          tma_load_3d(base + C::OFF_V + bx * C::BOX_BYTES, &tmV, bars.kv_full(), bx * 64, j * BT, bkv);
         }
-        mbar_arrive_expect_tx(bars.do_full(st), C::TILE_BYTES);
-        for (int bx = 0; bx < C::BOXES; ++bx)
-          tma_load_3d(base + C::OFF_DO + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmdO, bars.do_full(st), bx * 64,
-                      i * BT, bhq);
-        issued = 2 * it + 2;
-      }
-      if (*abort) {
-        drain_wait(bars.kv_full(), 0);
-        for (int t = (issued > 4 ? issued - 4 : 0); t < issued; ++t) {
-          const int it = t >> 1;
-          const uint32_t bar = (t & 1) ? bars.do_full(it & 1) : bars.q_full(it & 1);
-          drain_wait(bar, (it >> 1) & 1);
+        int issued = 0;
+        QWalk qw(i0, T);
+        for (int it = 0; it < n_it; ++it, qw.next()) {
+          const int st = it & 1;
+          const uint32_t ph = (it >> 1) & 1;
+          const int bhq = bhq0 + qw.head;
+          const int i = qw.tile;
+          if (!mbar_wait_sleep(bars.q_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 1)) break;
+          mbar_arrive_expect_tx(bars.q_full(st), C::TILE_BYTES + 1024);
+          for (int bx = 0; bx < C::BOXES; ++bx)
+            tma_load_3d(base + C::OFF_Q + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, bars.q_full(st), bx * 64,
+                        i * BT, bhq);
+          const long long voff = static_cast<long long>(bhq) * p.Npad + i * BT;
+          bulk_load_1d(base + C::OFF_VEC + st * 1024, p.neg_lse2 + voff, 512, bars.q_full(st));
+          bulk_load_1d(base + C::OFF_VEC + st * 1024 + 512, p.delta + voff, 512, bars.q_full(st));
+          if (!mbar_wait_sleep(bars.do_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 2)) {
+            issued = 2 * it + 1;
+            break;
+          }
+          mbar_arrive_expect_tx(bars.do_full(st), C::TILE_BYTES);
+          for (int bx = 0; bx < C::BOXES; ++bx)
+            tma_load_3d(base + C::OFF_DO + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmdO, bars.do_full(st), bx * 64,
+                        i * BT, bhq);
+          issued = 2 * it + 2;
+        }
+        if (*abort) {
+          drain_wait(bars.kv_full(), 0);
+          for (int t = (issued > 4 ? issued - 4 : 0); t < issued; ++t) {
+            const int it = t >> 1;
+            const uint32_t bar = (t & 1) ? bars.do_full(it & 1) : bars.q_full(it & 1);
+            drain_wait(bar, (it >> 1) & 1);
+          }
         }
       }
-    }
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      constexpr uint32_t IDESC_SS = idesc_bf16(BT, BT, false, false);
-      constexpr uint32_t IDESC_TS = idesc_bf16(BT, D, false, true);
-      constexpr uint32_t IDESC_DQ = idesc_bf16(BT, D, true, true);
-      const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
-      bool ok = mbar_wait_sleep(bars.kv_full(), 0, abort, p.status, SITE_BWD + 3);
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        const uint32_t sQ = base + C::OFF_Q + st * C::TILE_BYTES;
-        const uint32_t sdO = base + C::OFF_DO + st * C::TILE_BYTES;
-        if (!mbar_wait_sleep(bars.q_full(st), ph, abort, p.status, SITE_BWD + 4)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K_j Q_i^T
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + C::COL_S, smem_desc_sw128(sK + off, 16, 1024), smem_desc_sw128(sQ + off, 16, 1024),
-                 IDESC_SS, kk > 0 ? 1u : 0u);
+    } else if (warp == MMA_WARP) {
+      // ------------------------------------------------------------ MMA issue
+      if (lane == 0) {
+        constexpr uint32_t IDESC_SS = idesc_bf16(BT, BT, false, false);
+        constexpr uint32_t IDESC_TS = idesc_bf16(BT, D, false, true);
+        constexpr uint32_t IDESC_DQ = idesc_bf16(BT, D, true, true);
+        const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
+        bool ok = mbar_wait_sleep(bars.kv_full(), 0, abort, p.status, SITE_BWD + 3);
+        for (int it = 0; ok && it < n_it; ++it) {
+          const int st = it & 1;
+          const uint32_t ph = (it >> 1) & 1;
+          const uint32_t sQ = base + C::OFF_Q + st * C::TILE_BYTES;
+          const uint32_t sdO = base + C::OFF_DO + st * C::TILE_BYTES;
+          if (!mbar_wait_sleep(bars.q_full(st), ph, abort, p.status, SITE_BWD + 4)) break;
+          tc_fence_after();
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K_j Q_i^T
+            const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+            mma_ss(tmem + C::COL_S, smem_desc_sw128(sK + off, 16, 1024), smem_desc_sw128(sQ + off, 16, 1024),
+                   IDESC_SS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bars.s_full());
+          if (!mbar_wait_sleep(bars.do_full(st), ph, abort, p.status, SITE_BWD + 5)) break;
+          if (C::DQ_SHARES_DP && it > 0 && !mbar_wait_sleep(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
+            break;
+          tc_fence_after();
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V_j dO_i^T
+            const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+            mma_ss(tmem + C::COL_DP, smem_desc_sw128(sV + off, 16, 1024), smem_desc_sw128(sdO + off, 16, 1024),
+                   IDESC_SS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bars.dp_full());
+          if (!mbar_wait_sleep(bars.p_ready(), it & 1, abort, p.status, SITE_BWD + 7)) break;
+          tc_fence_after();
+  #pragma unroll
+          for (int kk = 0; kk < BT / 16; ++kk)  // dV += P^T dO_i
+            mma_ts(tmem + C::COL_DV, tmem + C::COL_S + (kk >> 2) * 64 + (kk & 3) * 8,
+                   smem_desc_sw128(sdO + kk * 2048, C::BOX_BYTES, 1024),
+                   IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bars.dv_done());
+          if (!mbar_wait_sleep(bars.dst_ready(), it & 1, abort, p.status, SITE_BWD + 8)) break;
+          tc_fence_after();
+  #pragma unroll
+          for (int kk = 0; kk < BT / 16; ++kk)  // dK += dS^T Q_i
+            mma_ts(tmem + C::COL_DK, tmem + C::COL_S + (kk >> 2) * 64 + 32 + (kk & 3) * 8,
+                   smem_desc_sw128(sQ + kk * 2048, C::BOX_BYTES, 1024),
+                   IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bars.q_empty(st));
+          if (!mbar_wait_sleep(bars.dss_ready(), it & 1, abort, p.status, SITE_BWD + 16)) break;
+          if (!C::DQ_SHARES_DP && it > 0 &&
+              !mbar_wait_sleep(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
+            break;
+          tc_fence_after();
+          const uint32_t sdS = ds_smem(st);
+  #pragma unroll
+          for (int kk = 0; kk < BT / 16; ++kk)  // dQ_i = dS K_j (A and B MN-major)
+            mma_ss(tmem + C::COL_DQ, smem_desc_sw128(sdS + kk * 2048, 16384, 1024),
+                   smem_desc_sw128(sK + kk * 2048, C::BOX_BYTES, 1024), IDESC_DQ, kk > 0 ? 1u : 0u);
+          mma_commit(bars.dq_full());
+          mma_commit(bars.do_empty(st));
         }
-        mma_commit(bars.s_full());
-        if (!mbar_wait_sleep(bars.do_full(st), ph, abort, p.status, SITE_BWD + 5)) break;
-        if (C::DQ_SHARES_DP && it > 0 && !mbar_wait_sleep(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
-          break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V_j dO_i^T
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + C::COL_DP, smem_desc_sw128(sV + off, 16, 1024), smem_desc_sw128(sdO + off, 16, 1024),
-                 IDESC_SS, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bars.dp_full());
-        if (!mbar_wait_sleep(bars.p_ready(), it & 1, abort, p.status, SITE_BWD + 7)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk)  // dV += P^T dO_i
-          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, smem_desc_sw128(sdO + kk * 2048, C::BOX_BYTES, 1024),
-                 IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bars.dv_done());
-        if (!mbar_wait_sleep(bars.dst_ready(), it & 1, abort, p.status, SITE_BWD + 8)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk)  // dK += dS^T Q_i
-          mma_ts(tmem + C::COL_DK, tmem + C::COL_S + 64 + kk * 8, smem_desc_sw128(sQ + kk * 2048, C::BOX_BYTES, 1024),
-                 IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bars.q_empty(st));
-        if (!mbar_wait_sleep(bars.dss_ready(), it & 1, abort, p.status, SITE_BWD + 16)) break;
-        if (!C::DQ_SHARES_DP && it > 0 &&
-            !mbar_wait_sleep(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
-          break;
-        tc_fence_after();
-        const uint32_t sdS = ds_smem(st);
-#pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk)  // dQ_i = dS K_j (A and B MN-major)
-          mma_ss(tmem + C::COL_DQ, smem_desc_sw128(sdS + kk * 2048, 16384, 1024),
-                 smem_desc_sw128(sK + kk * 2048, C::BOX_BYTES, 1024), IDESC_DQ, kk > 0 ? 1u : 0u);
-        mma_commit(bars.dq_full());
-        mma_commit(bars.do_empty(st));
+        mma_commit(bars.dkdv_done());
       }
-      mma_commit(bars.dkdv_done());
-    }
-  } else if (warp < 4) {
+    }  // warps 14, 15: no role
+  } else if (warp < 8) {
     // ------------------------------------------------------------ P and dS (thread = key row)
-    const int r = warp * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::COL_S;
-    const uint32_t tDP = tmem + lane_off + C::COL_DP;
+    // warpgroups 0 and 1, 64 query columns each
+    setmaxnreg_inc<REGS_COMPUTE>();
+    const int half = warp >> 2;  // query columns [64 half, 64 half + 64) of S^T and dP^T
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::COL_S + 64 * half;  // S^T; then P^T at +0, dS^T at +32
+    const uint32_t tDP = tmem + lane_off + C::COL_DP + 64 * half;
     const float cl2 = p.scale_log2;
     bool ok = true;
     QWalk qw(i0, T);
@@ -357,19 +379,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.s_full(), it & 1, abort, p.status, SITE_BWD + 10));
       if (!ok) break;
       tc_fence_after();
-      const float* vec_lse = reinterpret_cast<const float*>(base_ptr + C::OFF_VEC + st * 1024);
-      const float* vec_d = vec_lse + 128;
-      // P^T in two halves of 64 queries (keeps the live registers low): the
-      // packed bf16 P^T of queries 64h.. lands in columns 32h.. of S^T, which
-      // this thread has already read
-      const int qlim = p.N - i * BT;  // queries past N are padding
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      const float* vec = reinterpret_cast<const float*>(base_ptr + C::OFF_VEC + st * 1024);
+      const float* vec_lse = vec + 64 * half;
+      const float* vec_d = vec + 128 + 64 * half;
+      const int qlim = p.N - i * BT - 64 * half;  // queries of this half past N are padding
+      {
         float s[64];
         {
           uint32_t t[2][32];
-          tmem_ld_x32(tS + 64 * h, t[0]);
-          tmem_ld_x32(tS + 64 * h + 32, t[1]);
+          tmem_ld_x32(tS, t[0]);
+          tmem_ld_x32(tS + 32, t[1]);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 2; ++c)
@@ -378,7 +397,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         }
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(vec_lse + 64 * h + c);
+          const float4 l4 = *reinterpret_cast<const float4*>(vec_lse + c);
           s[c] = ex2(fmaf(s[c], cl2, l4.x));
           s[c + 1] = ex2(fmaf(s[c + 1], cl2, l4.y));
           s[c + 2] = ex2(fmaf(s[c + 2], cl2, l4.z));
@@ -387,18 +406,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         if (CAUSAL && i == j) {  // diagonal tile: key r sees queries >= r
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (64 * h + c < r) s[c] = 0.f;
+            if (64 * half + c < r) s[c] = 0.f;
         }
-        if (qlim < BT) {
+        if (qlim < 64) {
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (64 * h + c >= qlim) s[c] = 0.f;
+            if (c >= qlim) s[c] = 0.f;
         }
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[2 * e], s[2 * e + 1]);
-        tmem_st_x16(tS + 32 * h, *reinterpret_cast<const uint32_t(*)[16]>(pk));
-        tmem_st_x16(tS + 32 * h + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
+        tmem_st_x16(tS, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+        tmem_st_x16(tS + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -411,9 +430,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       // dS = P (dP - D), 32 queries at a time with P^T read back from tensor
       // memory: into tensor memory first (dK can start at once), then into
       // shared memory once dV has finished reading this dO slot (dQ)
-      uint32_t dsk[64];
+      uint32_t dsk[32];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t t[32], pp[16];
         tmem_ld_x32(tDP + cc * 32, t);
         tmem_ld_x16(tS + cc * 16, pp);
@@ -425,7 +444,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           dsk[cc * 16 + e] = pack_bf16x2(bf16_lo(pp[e]) * (__uint_as_float(t[2 * e]) - dd.x),
                                          bf16_hi(pp[e]) * (__uint_as_float(t[2 * e + 1]) - dd.y));
         }
-        tmem_st_x16(tS + 64 + cc * 16, *reinterpret_cast<const uint32_t(*)[16]>(dsk + cc * 16));
+        tmem_st_x16(tS + 32 + cc * 16, *reinterpret_cast<const uint32_t(*)[16]>(dsk + cc * 16));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -433,23 +452,21 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (lane == 0) mbar_arrive(bars.dst_ready());
       ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.dv_done(), it & 1, abort, p.status, SITE_BWD + 12));
       if (!ok) break;
-      const uint32_t sdS = ds_smem(st);
+      const uint32_t box = ds_smem(st) + half * C::BOX_BYTES;  // queries [64 half, 64 half + 64)
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t addr = sdS + (cc >> 1) * C::BOX_BYTES + sw128_offset(r, (cc & 1) * 4 + q);
-          const int e = cc * 16 + 4 * q;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dsk[e]), "r"(dsk[e + 1]),
-                       "r"(dsk[e + 2]), "r"(dsk[e + 3])
-                       : "memory");
-        }
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t addr = box + sw128_offset(r, ch);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dsk[4 * ch]), "r"(dsk[4 * ch + 1]),
+                     "r"(dsk[4 * ch + 2]), "r"(dsk[4 * ch + 3])
+                     : "memory");
+      }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.dss_ready());
     }
     // ------------------------------------------------------------ dK, dV epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.dkdv_done(), 0, abort, p.status, SITE_BWD + 13));
+    if (half == 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.dkdv_done(), 0, abort, p.status, SITE_BWD + 13));
+    if (half != 0) ok = false;  // warpgroup 0 writes dK and dV
     if (ok) {
       tc_fence_after();
       for (int which = 0; which < 2; ++which) {
@@ -486,8 +503,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         bulk_wait_read0();
       }
     }
-  } else if (warp < 8) {
+  } else {
     // ------------------------------------------------------------ dQ drain (thread = query row)
+    // warpgroup 2
+    setmaxnreg_inc<REGS_DRAIN>();
     const int w = warp & 3;
     const uint32_t tDQ = tmem + (static_cast<uint32_t>(w * 32) << 16) + C::COL_DQ;
     const uint32_t stg0 = base + C::OFF_STG + w * 2 * 2048;
@@ -560,6 +579,16 @@ cudaError_t launch_main(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CU
                         const CUtensorMap& tmdQacc, const BwdParams& p, int B, cudaStream_t stream) {
   using C = BwdCfg<D>;
   auto kern = bwd_bf16_kernel<D, CAUSAL>;
+  // the setmaxnreg increases wait until the CTA's register pool has room:
+  // make sure the compiled launch allocation covers the split
+  static int regs = 0;
+  if (regs == 0) {
+    cudaFuncAttributes fa_attr;
+    cudaError_t e0 = cudaFuncGetAttributes(&fa_attr, kern);
+    if (e0 != cudaSuccess) return e0;
+    regs = fa_attr.numRegs;
+  }
+  if (256 * REGS_COMPUTE + 128 * REGS_DRAIN + 128 * REGS_OTHER > BWD_THREADS * regs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(B * p.Hkv * p.num_tiles);
