@@ -30,3 +30,9 @@ from .fp8 import (  # noqa: F401
     fp8_attention_forward,
     naive_fp8_attention_forward,
 )
+from .mxfp8 import (  # noqa: F401
+    mx_quantize,
+    mx_dequantize,
+    mx_roundtrip,
+    mxfp8_attention_forward,
+)
