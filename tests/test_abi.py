@@ -139,3 +139,17 @@ def test_decode_rejects_bad_arguments(lib):
     assert lib.fa_decode_workspace_size(2, 8, 1, 4, 4096, 128, 0) == 0
     # the workspace holds partial rows per split, not an Nq x Nk matrix
     assert lib.fa_decode_workspace_size(16, 32, 8, 1, 131072, 128, 0) < 64 * 2 ** 20
+
+
+def test_decode_workspace_matches_the_documented_layout(lib):
+    """slots = min(CTAs, units) + B*Hkv with the automatic CTA count sized for
+    at most 1024; partial rows (d floats) then partial LSEs, each region rounded
+    up to 256 bytes. Device independent, so it holds without a GPU."""
+    up = lambda x: (x + 255) // 256 * 256
+    for B, Hq, Hkv, Nq, Nk, d, ctas in [(16, 32, 8, 1, 16384, 128, 0), (1, 4, 1, 4, 100, 64, 0),
+                                        (2, 8, 2, 2, 3000, 128, 7), (2, 8, 2, 2, 3000, 128, 100000),
+                                        (64, 8, 8, 1, 64, 128, 0)]:
+        R = (Hq // Hkv) * Nq
+        units = B * Hkv * ((Nk + 63) // 64)
+        slots = min(ctas if ctas > 0 else 1024, units) + B * Hkv
+        assert lib.fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, ctas) == up(slots * R * d * 4) + up(slots * R * 4)
