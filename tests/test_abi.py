@@ -153,3 +153,26 @@ def test_decode_workspace_matches_the_documented_layout(lib):
         units = B * Hkv * ((Nk + 63) // 64)
         slots = min(ctas if ctas > 0 else 1024, units) + B * Hkv
         assert lib.fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, ctas) == up(slots * R * d * 4) + up(slots * R * 4)
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/fa.h compiles as C99 and a C program linked against the library
+    sees the declared behaviour of the host-side entry points."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    from exact_tiled_attention_42_b200 import _lib
+    cuda_inc = next((p for p in ("/usr/local/cuda/include",) if os.path.isdir(p)), None)
+    if cuda_inc is None:
+        pytest.skip("no CUDA headers")
+    exe = tmp_path / "c_abi_check"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    cmd = [gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc,
+           os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", str(exe), "-L", libdir, "-l:libfa_b200.so",
+           "-Wl,-rpath," + libdir]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "ok"
