@@ -1,0 +1,63 @@
+"""The FP8 oracle's pins catch plausible mistakes: each case plants one error
+in a copy of oracle/fp8.py (never in the oracle itself), swaps the copy's
+functions into the ``oracle`` package, and expects at least one named pin to
+fail."""
+
+import importlib.util
+import os
+import sys
+
+import pytest
+
+import oracle
+import oracle.fp8 as fp8mod
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+import test_oracle_fp8_pins as pins  # noqa: E402
+
+SRC = open(fp8mod.__file__).read()
+
+MUTATIONS = [
+    ("ties away from zero", "r = np.round(ax / quantum) * quantum", "r = np.floor(ax / quantum + 0.5) * quantum",
+     [pins.test_e4m3_ties_go_to_even_and_saturate, pins.test_e4m3_round_matches_torch_in_range]),
+    ("no saturation", "r = np.minimum(r, E4M3_MAX)", "r = r",
+     [pins.test_e4m3_ties_go_to_even_and_saturate]),
+    ("block scale inverted", "scales[..., bi] = np.where(nz, safe / np.float32(E4M3_MAX)",
+     "scales[..., bi] = np.where(nz, np.float32(E4M3_MAX) / safe", [pins.test_block_quantize_properties]),
+    ("sign vector ignored", "return (x * sigma) @ hadamard(x.shape[-1])", "return x @ hadamard(x.shape[-1])",
+     [pins.test_rotation_preserves_scores_up_to_d]),
+    ("rotation's 1/d not folded", "sfac = scale / d", "sfac = scale",
+     [lambda: pins.test_fp8_emulation_within_e4m3_error_of_exact(True)]),
+    ("V's block scale not folded into P", "wkey = _expand_rows(vs[b, kvh], N, block_rows) / vref * p_lift",
+     "wkey = np.full(N, p_lift)",
+     [lambda: pins.test_fp8_emulation_within_e4m3_error_of_exact(False)]),
+    ("O not rescaled when the max grows", "acc = acc * alpha[:, None] + pq @ vv[b, kvh, j0:j1].astype(np.float64)",
+     "acc = acc + pq @ vv[b, kvh, j0:j1].astype(np.float64)",
+     [lambda: pins.test_fp8_emulation_within_e4m3_error_of_exact(False)]),
+]
+
+SWAPPED = ("hadamard", "rotate_rows", "e4m3_round", "e4m3_encode", "e4m3_decode", "block_quantize",
+           "fp8_attention_forward", "naive_fp8_attention_forward")
+
+
+def _mutated_module(old, new):
+    assert SRC.count(old) == 1, old
+    spec = importlib.util.spec_from_loader("fp8_mutant", loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    exec(compile(SRC.replace(old, new), "fp8_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new,catchers", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_planted_mistake(monkeypatch, name, old, new, catchers):
+    mod = _mutated_module(old, new)
+    for fn in SWAPPED:
+        monkeypatch.setattr(oracle, fn, getattr(mod, fn))
+    caught = 0
+    for pin in catchers:
+        try:
+            pin()
+        except AssertionError:
+            caught += 1
+    assert caught > 0, f"no pin caught the planted mistake: {name}"
