@@ -23,6 +23,7 @@
 // accumulator) at the start of each call. Calls whose executions overlap on
 // the GPU (different streams, or different host threads with no ordering
 // between them) race on the array and give wrong results: serialise them.
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -51,16 +52,27 @@ void* scratch_ptr() {
   return g_scratch_ptr[dev];
 }
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 }  // namespace
 
 extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                                     const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N,
                                     int d, int causal, float scale, cudaStream_t stream) {
+  // Argument errors first, in fa_bwd's order (null pointers, sizes, alignment),
+  // so a call that is wrong in several ways reports the same error as fa_bwd;
+  // only then the size limit of the built-in scratch.
+  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!ptr) return FA_ERR_INVALID_ARG;
   const size_t need = fa_bwd_workspace_size(B, Hq, Hkv, N, d);
   if (need == 0) {
     // Invalid sizes: let fa_bwd's own checks report the precise error.
     return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, nullptr, 0, B, Hq, Hkv, N, d, causal, scale, stream);
   }
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
   if (need > FA_BWD_NOALLOC_MAX_BYTES) return FA_ERR_WORKSPACE;  // problem too large for the built-in scratch
   void* ws = scratch_ptr();
   if (!ws) return FA_ERR_CUDA;

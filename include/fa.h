@@ -87,8 +87,12 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  cudaStream_t stream);
 
 /*
- * Largest scratch, in bytes, that fa_bwd_noalloc can use (32 MiB). It is
- * enough for B*Hq*N up to about 63,000 query rows at d = 128 (126,000 at d = 64).
+ * Largest scratch, in bytes, that fa_bwd_noalloc can use (32 MiB). A problem
+ * fits when fa_bwd_workspace_size(B, Hq, Hkv, N, d) <= FA_BWD_NOALLOC_MAX_BYTES.
+ * The scratch holds 8 bytes per query row padded to Npad = 128 * ceil(N / 128)
+ * rows per head, plus 4 * d bytes per real query row, so about 64,500 query
+ * rows (B * Hq * N) at d = 128 and 127,000 at d = 64 when N is a multiple of
+ * 128, and fewer when padding is a large share of N (small or ragged N).
  */
 #define FA_BWD_NOALLOC_MAX_BYTES (32u * 1024u * 1024u)
 
@@ -103,7 +107,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * that must not call cudaMalloc/cudaFree there because they synchronise the
  * device). Arguments, layouts and results are those of fa_bwd.
  *   - Allocates nothing: no cudaMalloc, no cudaFree.
- *   - Returns FA_ERR_WORKSPACE, launching nothing, when fa_bwd_workspace_size
+ *   - Argument errors are reported as fa_bwd reports them (null pointer,
+ *     invalid size or scale, misalignment, checked in that order); after
+ *     them, FA_ERR_WORKSPACE, launching nothing, when fa_bwd_workspace_size
  *     for these sizes exceeds FA_BWD_NOALLOC_MAX_BYTES.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.

@@ -27,6 +27,7 @@ from .fp8 import (  # noqa: F401
     e4m3_encode,
     e4m3_decode,
     block_quantize,
+    per_tensor_quantize,
     fp8_attention_forward,
     naive_fp8_attention_forward,
 )

@@ -24,13 +24,22 @@ rotation. Readings used here:
   e4m3; the 256 and max(sV) are undone at the end. This folds V's per-block
   scale into P; w <= 256 keeps P w below 448.
 * Baseline FP8: one amax scale per tensor for each of Q, K and V, no rotation,
-  exact softmax, then the normalised P rounded to e4m3.
+  exact softmax with the row's final maximum, and the unnormalised P~ =
+  exp(S - m) rounded to e4m3 with no scale factor (the quantity a tiled
+  kernel multiplies by V; the division by the row sum comes once at the
+  end). Rounding the normalised probabilities instead is kept as an option:
+  at large N most of them fall below e4m3's subnormals, which would make the
+  baseline look far worse than a real FP8 kernel.
 
 Parity pins: ``e4m3_round`` against torch's float8_e4m3fn conversion for
 in-range values; ``hadamard`` by orthogonality and the Sylvester recursion;
 ``block_quantize`` by the largest element mapping to 448 and a half-quantum
-error bound; ``fp8_attention_forward`` and ``naive_fp8_attention_forward``
-against exact attention within the error bound of e4m3 rounding. The ratio of
+error bound; ``fp8_attention_forward`` against exact attention within the
+error bound of e4m3 rounding, and against its own single-tile reading (P
+rounded against the row's final maximum) within two half-quanta of P;
+``per_tensor_quantize`` and ``naive_fp8_attention_forward`` by closed forms
+on inputs already on the e4m3 grid (hand-computed codes of P, both P forms,
+per-tensor rather than per-head scales). The ratio of
 FP8 errors the abstract reports (2.6x) is parity unpinned: it is reported, not
 asserted.
 """
@@ -184,41 +193,59 @@ def fp8_attention_forward(q, k, v, causal: bool, scale: float, sigma=None,
     return o, lse
 
 
-def naive_fp8_attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int = 2048, heads=None):
-    """Baseline FP8: per-tensor amax scales for Q, K, V, no rotation, exact
-    softmax, normalised P rounded to e4m3. Returns O. Query rows are formed
-    ``row_chunk`` at a time (each row still sees all of its keys). ``heads``,
-    a list of (b, h), limits which heads' outputs are computed (the others
-    are NaN); the scales still come from the whole tensors."""
-    def per_tensor(x):
-        x32 = np.asarray(x, np.float64).astype(np.float32)
-        amax = np.float32(np.max(np.abs(x32)))
-        if amax == 0:
-            return x32.astype(np.float64)
-        inv = np.float32(E4M3_MAX) / amax
-        s = amax / np.float32(E4M3_MAX)
-        return e4m3_round((x32 * inv).astype(np.float32)).astype(np.float64) * float(s)
+def per_tensor_quantize(x):
+    """One e4m3 scale for the whole tensor: s = amax / 448 (1 when amax = 0),
+    codes e4m3(x * (448 / amax)) decided in float32. Returns (values on the
+    e4m3 grid as float64, s)."""
+    x32 = np.asarray(x, np.float64).astype(np.float32)
+    amax = np.max(np.abs(x32)).astype(np.float32)
+    nz = amax > 0
+    safe = np.where(nz, amax, np.float32(1.0)).astype(np.float32)
+    inv = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(1.0)).astype(np.float32)
+    s = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float64)
+    return e4m3_round((x32 * inv).astype(np.float32)).astype(np.float64), s
 
-    qh, kh = per_tensor(q), per_tensor(k)
-    vq = np.asarray(v, np.float64).astype(np.float32)
-    vamax = np.float32(np.max(np.abs(vq)))
-    vinv = np.float32(E4M3_MAX) / vamax
-    vvals = e4m3_round((vq * vinv).astype(np.float32)).astype(np.float64)
-    vscale = float(vamax / np.float32(E4M3_MAX))
+
+def naive_fp8_attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int = 2048, heads=None,
+                                p_form: str = "unnormalised"):
+    """Baseline FP8 attention: one amax scale per tensor for each of Q, K and
+    V, no rotation, exact softmax with the row's final maximum, and P rounded
+    to e4m3 with no extra scale factor. ``p_form`` says which P is rounded:
+
+    * "unnormalised" (the baseline reported): P~ = exp(S - m) in (0, 1], the
+      quantity a tiled kernel feeds to its P V product (the division by the
+      row sum comes once at the end), so O = (e4m3(P~) V) / sum_j P~.
+    * "normalised": the softmax probabilities exp(S - m) / sum_j exp(S - m)
+      themselves, O = e4m3(P) V. At large N most of them fall below e4m3's
+      subnormal range and round to zero, so this form is far less accurate.
+
+    Returns O. Query rows are formed ``row_chunk`` at a time (each row still
+    sees all of its keys). ``heads``, a list of (b, h), limits which heads'
+    outputs are computed (the others are NaN); the scales still come from the
+    whole tensors."""
+    if p_form not in ("unnormalised", "normalised"):
+        raise ValueError(p_form)
+    qv, qs = per_tensor_quantize(q)
+    kv_, ks = per_tensor_quantize(k)
+    vv, vs = per_tensor_quantize(v)
+    qh, kh = qv * qs, kv_ * ks
+    vs = np.broadcast_to(vs, vv.shape[:2] + (1, 1))   # one value per (b, kv head): the tensor's scale
     B, Hq, N, d = qh.shape
     g = Hq // kh.shape[1]
     o = np.full((B, Hq, N, d), np.nan)
     todo = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else list(heads)
     for b, h in todo:
-        if True:
-            for r0 in range(0, N, row_chunk):
-                r1 = min(N, r0 + row_chunk)
-                s = scale * (qh[b, h, r0:r1] @ kh[b, h // g].T)
-                if causal:
-                    s = np.where(np.arange(N)[None, :] > np.arange(r0, r1)[:, None], -np.inf, s)
-                m = np.max(s, axis=1, keepdims=True)
-                e = np.exp(s - m)
-                p = e / e.sum(axis=1, keepdims=True)
-                pq = e4m3_round(p.astype(np.float32)).astype(np.float64)
-                o[b, h, r0:r1] = (pq @ vvals[b, h // g]) * vscale
+        for r0 in range(0, N, row_chunk):
+            r1 = min(N, r0 + row_chunk)
+            s = scale * (qh[b, h, r0:r1] @ kh[b, h // g].T)
+            if causal:
+                s = np.where(np.arange(N)[None, :] > np.arange(r0, r1)[:, None], -np.inf, s)
+            e = np.exp(s - np.max(s, axis=1, keepdims=True))
+            l = e.sum(axis=1, keepdims=True)
+            if p_form == "normalised":
+                pq = e4m3_round((e / l).astype(np.float32)).astype(np.float64)
+                o[b, h, r0:r1] = (pq @ vv[b, h // g]) * vs[b, h // g]
+            else:
+                pq = e4m3_round(e.astype(np.float32)).astype(np.float64)
+                o[b, h, r0:r1] = (pq @ vv[b, h // g]) * vs[b, h // g] / l
     return o

@@ -86,6 +86,28 @@ def test_bwd_rejects_bad_arguments(lib):
     assert bwd(dq=P + 2) == 3
 
 
+def test_bwd_noalloc_reports_argument_errors_before_its_size_limit(lib):
+    """fa_bwd_noalloc checks arguments in fa_bwd's order before the size of
+    its built-in scratch: a call that is too large and also wrong in another
+    way reports the other error. Sizes: 2 x 32 heads x 8192 rows x 128 needs
+    far more than FA_BWD_NOALLOC_MAX_BYTES."""
+    big = (2, 32, 8, 8192, 128)
+    def nb(dq=P, scale=0.088, sizes=big):
+        return lib.fa_bwd_noalloc(P, P, P, P, P, P, dq, P, P, *sizes, 1, scale, None)
+    assert lib.fa_bwd_workspace_size(*big) > 32 * 1024 * 1024
+    assert nb(dq=None) == 1                    # null pointer
+    assert nb(scale=0.0) == 1                  # bad scale
+    assert nb(scale=float("nan")) == 1
+    assert nb(sizes=(2, 33, 8, 8192, 128)) == 1  # Hq % Hkv != 0
+    assert nb(sizes=(2, 32, 8, 8192, 96)) == 2   # head dimension
+    assert nb(dq=P + 2) == 3                   # misaligned
+    assert nb() == 4                           # only then: larger than the built-in scratch
+    # the limit is exact: 2 x 64 heads x 992 rows x 64 needs exactly 32 MiB
+    # (launching would need a GPU, so only the size query is checked here)
+    assert lib.fa_bwd_workspace_size(2, 64, 16, 992, 64) == 32 * 1024 * 1024
+    assert lib.fa_bwd_workspace_size(1, 129, 129, 992, 64) > 32 * 1024 * 1024
+
+
 def test_fp8_rejects_bad_arguments(lib):
     ws = lib.fa_fp8_workspace_size(1, 2, 2, 128, 128)
     assert ws > 0

@@ -35,10 +35,32 @@ MUTATIONS = [
     ("O not rescaled when the max grows", "acc = acc * alpha[:, None] + pq @ vv[b, kvh, j0:j1].astype(np.float64)",
      "acc = acc + pq @ vv[b, kvh, j0:j1].astype(np.float64)",
      [lambda: pins.test_fp8_emulation_within_e4m3_error_of_exact(False)]),
+    ("emulated P not rounded", "pq = e4m3_round((p * wkey[None, j0:j1]).astype(np.float32)).astype(np.float64)",
+     "pq = p * wkey[None, j0:j1]",
+     [lambda: pins.test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(128, False)]),
+    ("emulated P rounded against a stale max", "p = np.exp2(s - m_new[:, None])", "p = np.exp2(s - np.maximum(m, -60.0)[:, None])",
+     [lambda: pins.test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(128, False),
+      lambda: pins.test_fp8_emulation_within_e4m3_error_of_exact(False)]),
+    ("naive: P not rounded", "pq = e4m3_round(e.astype(np.float32)).astype(np.float64)", "pq = e",
+     [pins.test_naive_fp8_two_key_closed_form_unnormalised,
+      lambda: pins.test_naive_fp8_within_p_rounding_of_exact_on_grid("unnormalised")]),
+    ("naive: normalised P not rounded", "pq = e4m3_round((e / l).astype(np.float32)).astype(np.float64)",
+     "pq = e / l", [pins.test_naive_fp8_two_key_closed_form_normalised]),
+    ("naive: per-head instead of per-tensor amax", "amax = np.max(np.abs(x32)).astype(np.float32)",
+     "amax = np.max(np.abs(x32), axis=(-2, -1), keepdims=True).astype(np.float32)",
+     [pins.test_naive_fp8_two_key_closed_form_unnormalised]),
+    ("naive: V scale not applied", "o[b, h, r0:r1] = (pq @ vv[b, h // g]) * vs[b, h // g] / l",
+     "o[b, h, r0:r1] = (pq @ vv[b, h // g]) / l", [pins.test_naive_fp8_two_key_closed_form_unnormalised]),
+    ("naive: row sum of the rounded P", "o[b, h, r0:r1] = (pq @ vv[b, h // g]) * vs[b, h // g] / l",
+     "o[b, h, r0:r1] = (pq @ vv[b, h // g]) * vs[b, h // g] / pq.sum(axis=1, keepdims=True)",
+     [pins.test_naive_fp8_two_key_closed_form_unnormalised]),
+    ("per-tensor scale inverted", "s = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float64)",
+     "s = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(1.0)).astype(np.float64)",
+     [pins.test_per_tensor_quantize_closed_form]),
 ]
 
 SWAPPED = ("hadamard", "rotate_rows", "e4m3_round", "e4m3_encode", "e4m3_decode", "block_quantize",
-           "fp8_attention_forward", "naive_fp8_attention_forward")
+           "per_tensor_quantize", "fp8_attention_forward", "naive_fp8_attention_forward")
 
 
 def _mutated_module(old, new):

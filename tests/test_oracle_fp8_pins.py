@@ -157,3 +157,166 @@ def test_naive_head_subset_matches_full():
     part = oracle.naive_fp8_attention_forward(q, k, v, False, 0.125, heads=[(0, 2)])
     np.testing.assert_array_equal(part[0, 2], full[0, 2])
     assert np.isnan(part[0, 0]).all()
+
+
+# ---------------------------------------------------------------- the naive baseline
+
+def test_per_tensor_quantize_closed_form():
+    """Values already on the e4m3 grid times 2^-5, tensor amax 14 = 448 * 2^-5:
+    the scale is exactly 2^-5 and every code is the value / 2^-5."""
+    rng = np.random.default_rng(21)
+    codes = oracle.e4m3_round((rng.standard_normal((2, 3, 16, 8)) * 60).astype(np.float32)).astype(np.float64)
+    codes[0, 0, 0, 0] = 448.0
+    x = codes * 2.0 ** -5
+    vals, s = oracle.per_tensor_quantize(x)
+    assert s == 2.0 ** -5
+    np.testing.assert_array_equal(vals, codes)
+    z, s0 = oracle.per_tensor_quantize(np.zeros((1, 2, 3, 4)))
+    assert s0 == 1.0 and np.all(z == 0)
+
+
+def _two_key_case():
+    """Two heads, two keys, d = 4. Q and K put the scores at [0, ln 0.3] for
+    every query row (scale = -ln(0.3) / 448^2, K_1 = -448 e_0), so the
+    unnormalised P is [1, 0.3] and the probabilities [1/1.3, 0.3/1.3]. V of
+    head 0 lies on the e4m3 grid times 2^-5 with amax 14 (per-tensor scale
+    exactly 2^-5); V of head 1 is 0.05 / 0.1, which that scale does not
+    represent exactly."""
+    q = np.zeros((1, 2, 2, 4))
+    q[..., 0] = 448.0
+    k = np.zeros((1, 2, 2, 4))
+    k[:, :, 1, 0] = -448.0
+    v = np.zeros((1, 2, 2, 4))
+    v[0, 0, 0] = [14.0, -7.0, 3.5, 0.0]
+    v[0, 0, 1] = [7.0, 14.0, -14.0, 1.75]
+    v[0, 1, 0] = 0.05
+    v[0, 1, 1] = 0.1
+    scale = -math.log(0.3) / 448.0 ** 2
+    return q, k, v, scale
+
+
+def test_naive_fp8_two_key_closed_form_unnormalised():
+    """P~ = [1, 0.3]: e4m3(0.3) = 0.3125 (quantum 2^-5 in [0.25, 0.5), 9.6
+    quanta round to 10); O = (V_0 + 0.3125 V_1) / 1.3 with the row sum of the
+    unrounded P~. Head 1's V under the per-tensor scale 2^-5: 0.05 -> 1.6 ->
+    1.625 and 0.1 -> 3.2 -> 3.25 codes, i.e. 0.05078125 and 0.1015625 (a
+    per-head scale would have kept them nearly exact)."""
+    q, k, v, scale = _two_key_case()
+    o = oracle.naive_fp8_attention_forward(q, k, v, False, scale)
+    h0 = np.array([16.1875, -2.625, -0.875, 0.546875]) / 1.3
+    h1 = np.full(4, 0.05078125 + 0.3125 * 0.1015625) / 1.3
+    np.testing.assert_allclose(o[0, 0], np.stack([h0, h0]), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(o[0, 1], np.stack([h1, h1]), rtol=1e-12, atol=1e-12)
+    # causal: query row 0 sees key 0 alone (P~ = 1, exactly representable)
+    oc = oracle.naive_fp8_attention_forward(q, k, v, True, scale)
+    np.testing.assert_allclose(oc[0, 0, 0], v[0, 0, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(oc[0, 0, 1], h0, rtol=1e-12, atol=1e-12)
+
+
+def test_naive_fp8_two_key_closed_form_normalised():
+    """P = [1/1.3, 0.3/1.3] = [0.769.., 0.2307..]: e4m3 gives 0.75 (12.3
+    quanta of 2^-4) and 0.234375 (14.8 quanta of 2^-6 round to 15), and O =
+    0.75 V_0 + 0.234375 V_1 with no division."""
+    q, k, v, scale = _two_key_case()
+    o = oracle.naive_fp8_attention_forward(q, k, v, False, scale, p_form="normalised")
+    h0 = np.array([12.140625, -1.96875, -0.65625, 0.41015625])
+    h1 = np.full(4, 0.75 * 0.05078125 + 0.234375 * 0.1015625)
+    np.testing.assert_allclose(o[0, 0], np.stack([h0, h0]), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(o[0, 1], np.stack([h1, h1]), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("p_form", ["unnormalised", "normalised"])
+def test_naive_fp8_within_p_rounding_of_exact_on_grid(p_form):
+    """Q, K, V on the e4m3 grid with amax 448 quantise exactly, so only P's
+    rounding remains: each rounded entry is within half a quantum, at most
+    2^-4 of its value or 2^-10 in the subnormal range. Hence
+    |O - O_exact| <= 2^-4 (P |V|) + 2^-10 sum_j |V_j| / r, where r is the row
+    sum for the unnormalised form and 1 for the normalised one."""
+    rng = np.random.default_rng(22)
+    N, d = 96, 32
+    def grid():
+        x = oracle.e4m3_round((rng.standard_normal((1, 2, N, d)) * 30).astype(np.float32)).astype(np.float64)
+        x[0, 0, 0, 0] = 448.0
+        return x
+    q, k, v = grid(), grid(), grid()
+    scale = 1.0 / 8192
+    exact, lse = oracle.attention_forward(q, k, v, False, scale)
+    o = oracle.naive_fp8_attention_forward(q, k, v, False, scale, p_form=p_form)
+    s = scale * np.einsum("bhid,bhjd->bhij", q, k)
+    p = np.exp(s - lse[..., None])
+    r = np.exp(lse - s.max(-1)) if p_form == "unnormalised" else np.ones_like(lse)
+    bound = 2.0 ** -4 * (p @ np.abs(v)) + 2.0 ** -10 * np.abs(v).sum(-2)[..., None, :] / r[..., None]
+    assert np.all(np.abs(o - exact) <= bound * (1 + 1e-9) + 1e-12)
+    # and the rounding is really there: not equal to the exact result
+    assert np.max(np.abs(o - exact)) > 1e-3
+
+
+# ---------------------------------------------------------------- the emulation's P rounding, tile by tile
+
+def _dequantised(q, k, v, sigma, block_rows=64):
+    d = q.shape[-1]
+    if sigma is not None:
+        q, k = oracle.rotate_rows(q, sigma), oracle.rotate_rows(k, sigma)
+    out = []
+    for x in (q, k, v):
+        vals, sc = oracle.block_quantize(x, block_rows)
+        out.append(vals.astype(np.float64) * np.repeat(sc.astype(np.float64), block_rows, axis=-1)[..., :x.shape[-2], None])
+    return out, (1.0 / d if sigma is not None else 1.0)
+
+
+@pytest.mark.parametrize("tile", [16, 128, 1 << 20])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(tile, causal):
+    """With the operands' quantisation fixed, the FP8 emulation differs from
+    exact softmax attention on the dequantised Q, K, V only by P's e4m3
+    rounding. Per key j the rounded quantity is P~_j w_j, with P~_j <= 1 and
+    w_j = sV_j / max sV * 256; its half-quantum error is at most 2^-4 of it,
+    or 2^-10 below the normal range. In units of O that is at most
+    2^-4 P_ij |V^_jc| + 2^-10 |Vc_jc| (max sV / 256) / r_i, with P the exact
+    probabilities, V^ the dequantised V, Vc its codes and r_i the row's sum
+    exp(S - max S) (the running max only makes P~ larger, never the bound
+    smaller). The bound holds for every tile size, including a single tile
+    (P rounded against the row's final maximum), so the reading does not
+    depend on the kernel's 128-key schedule."""
+    q, k, v = _fp8_inputs(N=300, d=64, H=2, seed=23, outliers=0.003)
+    d = q.shape[-1]
+    scale = d ** -0.5
+    sigma = sign_vector(31, d)
+    (qh, kh, vh), fold = _dequantised(q, k, v, sigma)
+    exact_dq, lse = oracle.attention_forward(qh, kh, vh, causal, scale * fold)
+    o8, _ = oracle.fp8_attention_forward(q, k, v, causal, scale, sigma, tile=tile)
+    s = scale * fold * np.einsum("bhid,bhjd->bhij", qh, kh)
+    if causal:
+        s = np.where(np.triu(np.ones(s.shape[-2:], bool), 1), -np.inf, s)
+    p = np.exp(s - lse[..., None])
+    r = np.exp(lse - s.max(-1))
+    _, vs = oracle.block_quantize(v, 64)
+    vcodes, _ = oracle.block_quantize(v, 64)
+    sub = 2.0 ** -10 * (vs.max(-1) / 256.0)[..., None, None] * (np.abs(vcodes.astype(np.float64)).sum(-2)[..., None, :]
+                                                               / r[..., None])
+    bound = 2.0 ** -4 * (p @ np.abs(vh)) + sub
+    err = np.abs(o8 - exact_dq)
+    assert np.all(err <= bound * (1 + 1e-9) + 1e-12), float((err / bound).max())
+    assert err.max() > 1e-4  # P is really rounded
+
+
+def test_fp8_emulation_tile_schedule_moves_little():
+    """The 128-key tile schedule (P rounded against the running max) and a
+    single tile (P rounded against the final row max) round different
+    multiples of the same P, so they differ by at most two half-quanta per
+    term (the bound above, twice). Measured here: their RMS difference is a
+    small share of either reading's RMS error against exact attention."""
+    q, k, v = _fp8_inputs(N=512, d=128, H=2, seed=24, outliers=0.001)
+    d = q.shape[-1]
+    scale = d ** -0.5
+    sigma = sign_vector(32, d)
+    exact, _ = oracle.attention_forward(q, k, v, False, scale)
+    o128, _ = oracle.fp8_attention_forward(q, k, v, False, scale, sigma, tile=128)
+    o1, _ = oracle.fp8_attention_forward(q, k, v, False, scale, sigma, tile=1 << 20)
+    rms = lambda a: math.sqrt(np.mean(a ** 2))
+    (qh, kh, vh), fold = _dequantised(q, k, v, sigma)
+    _, lse = oracle.attention_forward(qh, kh, vh, False, scale * fold)
+    p = np.exp(scale * fold * np.einsum("bhid,bhjd->bhij", qh, kh) - lse[..., None])
+    assert np.all(np.abs(o128 - o1) <= 2 * 2.0 ** -4 * (p @ np.abs(vh)) + 1e-3)
+    assert rms(o128 - o1) <= 0.5 * min(rms(o128 - exact), rms(o1 - exact))
+    assert abs(rms(o128 - exact) - rms(o1 - exact)) <= 0.1 * rms(o1 - exact)
