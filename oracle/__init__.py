@@ -31,6 +31,7 @@ from .fp8 import (  # noqa: F401
     fp8_attention_forward,
     naive_fp8_attention_forward,
 )
+from .varlen import varlen_forward, varlen_backward  # noqa: F401
 from .mxfp8 import (  # noqa: F401
     mx_quantize,
     mx_dequantize,
