@@ -21,6 +21,7 @@ from .attention import (  # noqa: F401
 )
 from .fp8 import (  # noqa: F401
     E4M3_MAX,
+    FP8_TAU,
     hadamard,
     rotate_rows,
     e4m3_round,

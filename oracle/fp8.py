@@ -19,10 +19,12 @@ rotation. Readings used here:
   saturating. The quantised code is decided in float32, the precision the
   kernel uses: y is rounded once to float32, inv = 448 / amax and y * inv are
   single float32 operations, then rounded to e4m3.
-* P: within each 128-key tile, P = exp2(c S - m) with the exact running max
-  (P <= 1), multiplied by w = sV(key block) / max(sV) * 256 and rounded to
-  e4m3; the 256 and max(sV) are undone at the end. This folds V's per-block
-  scale into P; w <= 256 keeps P w below 448.
+* P: within each 128-key tile, P = exp2(c S - m) with a running max m that a
+  row raises only when the tile's max exceeds it by more than tau = 0.8
+  (log2 units; the same stale max enters the row sum and O, so the result is
+  the softmax's), multiplied by w = sV(key block) / max(sV) * 256 and rounded
+  to e4m3; the 256 and max(sV) are undone at the end. This folds V's
+  per-block scale into P; 2^0.8 * 256 = 445.7 keeps P w below 448.
 * Baseline FP8: one amax scale per tensor for each of Q, K and V, no rotation,
   exact softmax with the row's final maximum, and the unnormalised P~ =
   exp(S - m) rounded to e4m3 with no scale factor (the quantity a tiled
@@ -140,15 +142,23 @@ def _expand_rows(scales, N, block_rows):
     return np.repeat(np.asarray(scales, np.float64), block_rows, axis=-1)[..., :N]
 
 
+FP8_TAU = 0.8
+
+
 def fp8_attention_forward(q, k, v, causal: bool, scale: float, sigma=None,
-                          block_rows: int = 64, tile: int = 128, p_lift: float = 256.0):
+                          block_rows: int = 64, tile: int = 128, p_lift: float = 256.0, tau: float = FP8_TAU):
     """Emulate the FP8 forward (readings in the module docstring) in float64.
 
     Q and K are rotated with ``sigma`` (skipped when None), all three are block
     quantised, scores come from the dequantised operands, and keys are visited
-    ``tile`` at a time with an exact running max; P is rounded to e4m3 after
-    folding in V's block scale. Returns (O, LSE).
+    ``tile`` at a time. Each row keeps a running max that it raises to the
+    tile's max only when that exceeds it by more than ``tau`` (log2 units;
+    ``tau = 0`` is the exact running max), so P <= 2^tau; P is rounded to
+    e4m3 after folding in V's block scale (P w <= 2^tau * p_lift, below 448
+    for tau = 0.8, p_lift = 256). Returns (O, LSE).
     """
+    if 2.0 ** tau * p_lift > E4M3_MAX:
+        raise ValueError("2^tau * p_lift must stay within e4m3's range")
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
@@ -181,7 +191,8 @@ def fp8_attention_forward(q, k, v, causal: bool, scale: float, sigma=None,
                 s = c * (qh[b, h] @ kh[b, kvh, j0:j1].T)
                 if causal:
                     s = np.where(np.arange(j0, j1)[None, :] > np.arange(N)[:, None], -np.inf, s)
-                m_new = np.maximum(m, np.max(s, axis=1))
+                tmax = np.max(s, axis=1)
+                m_new = np.where(tmax > m + tau, np.maximum(m, tmax), m)
                 alpha = np.where(np.isneginf(m), 0.0, np.exp2(m - m_new))
                 p = np.exp2(s - m_new[:, None])
                 l = l * alpha + p.sum(axis=1)

@@ -37,10 +37,12 @@ MUTATIONS = [
      [lambda: pins.test_fp8_emulation_within_e4m3_error_of_exact(False)]),
     ("emulated P not rounded", "pq = e4m3_round((p * wkey[None, j0:j1]).astype(np.float32)).astype(np.float64)",
      "pq = p * wkey[None, j0:j1]",
-     [lambda: pins.test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(128, False)]),
+     [lambda: pins.test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(128, False, 0.8)]),
     ("emulated P rounded against a stale max", "p = np.exp2(s - m_new[:, None])", "p = np.exp2(s - np.maximum(m, -60.0)[:, None])",
-     [lambda: pins.test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(128, False),
+     [lambda: pins.test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(128, False, 0.8),
       lambda: pins.test_fp8_emulation_within_e4m3_error_of_exact(False)]),
+    ("max raised on every increase despite tau", "m_new = np.where(tmax > m + tau, np.maximum(m, tmax), m)",
+     "m_new = np.maximum(m, tmax)", [pins.test_fp8_deferred_max_two_tile_closed_form]),
     ("naive: P not rounded", "pq = e4m3_round(e.astype(np.float32)).astype(np.float64)", "pq = e",
      [pins.test_naive_fp8_two_key_closed_form_unnormalised,
       lambda: pins.test_naive_fp8_within_p_rounding_of_exact_on_grid("unnormalised")]),

@@ -264,9 +264,10 @@ def _dequantised(q, k, v, sigma, block_rows=64):
     return out, (1.0 / d if sigma is not None else 1.0)
 
 
+@pytest.mark.parametrize("tau", [0.0, 0.8])
 @pytest.mark.parametrize("tile", [16, 128, 1 << 20])
 @pytest.mark.parametrize("causal", [False, True])
-def test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(tile, causal):
+def test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(tile, causal, tau):
     """With the operands' quantisation fixed, the FP8 emulation differs from
     exact softmax attention on the dequantised Q, K, V only by P's e4m3
     rounding. Per key j the rounded quantity is P~_j w_j, with P~_j <= 1 and
@@ -277,14 +278,16 @@ def test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(tile
     exp(S - max S) (the running max only makes P~ larger, never the bound
     smaller). The bound holds for every tile size, including a single tile
     (P rounded against the row's final maximum), so the reading does not
-    depend on the kernel's 128-key schedule."""
+    depend on the kernel's 128-key schedule, and for a running max that is
+    raised only past tau = 0.8 (P up to 2^0.8, P w up to 445.7, still within
+    e4m3's normal range) as for the exact one."""
     q, k, v = _fp8_inputs(N=300, d=64, H=2, seed=23, outliers=0.003)
     d = q.shape[-1]
     scale = d ** -0.5
     sigma = sign_vector(31, d)
     (qh, kh, vh), fold = _dequantised(q, k, v, sigma)
     exact_dq, lse = oracle.attention_forward(qh, kh, vh, causal, scale * fold)
-    o8, _ = oracle.fp8_attention_forward(q, k, v, causal, scale, sigma, tile=tile)
+    o8, _ = oracle.fp8_attention_forward(q, k, v, causal, scale, sigma, tile=tile, tau=tau)
     s = scale * fold * np.einsum("bhid,bhjd->bhij", qh, kh)
     if causal:
         s = np.where(np.triu(np.ones(s.shape[-2:], bool), 1), -np.inf, s)
@@ -320,3 +323,53 @@ def test_fp8_emulation_tile_schedule_moves_little():
     assert np.all(np.abs(o128 - o1) <= 2 * 2.0 ** -4 * (p @ np.abs(vh)) + 1e-3)
     assert rms(o128 - o1) <= 0.5 * min(rms(o128 - exact), rms(o1 - exact))
     assert abs(rms(o128 - exact) - rms(o1 - exact)) <= 0.1 * rms(o1 - exact)
+
+
+def test_fp8_deferred_max_matches_the_exact_running_max():
+    """Raising a row's max only past tau rounds different multiples of the
+    same P (at most two half-quanta apart per term) and keeps the same
+    accuracy against exact attention; tau = 0 is the exact running max, whose
+    first tile sets m and whose P never exceeds 1."""
+    q, k, v = _fp8_inputs(N=640, d=128, H=2, seed=25, outliers=0.001)
+    d = q.shape[-1]
+    scale = d ** -0.5
+    sigma = sign_vector(33, d)
+    exact, lse = oracle.attention_forward(q, k, v, False, scale)
+    o0, l0 = oracle.fp8_attention_forward(q, k, v, False, scale, sigma, tau=0.0)
+    o8, l8 = oracle.fp8_attention_forward(q, k, v, False, scale, sigma, tau=0.8)
+    rms = lambda a: math.sqrt(np.mean(a ** 2))
+    (qh, kh, vh), fold = _dequantised(q, k, v, sigma)
+    _, lse_dq = oracle.attention_forward(qh, kh, vh, False, scale * fold)
+    p = np.exp(scale * fold * np.einsum("bhid,bhjd->bhij", qh, kh) - lse_dq[..., None])
+    assert np.all(np.abs(o0 - o8) <= 2 * 2.0 ** -4 * (p @ np.abs(vh)) + 1e-3)
+    assert abs(rms(o0 - exact) - rms(o8 - exact)) <= 0.1 * rms(o0 - exact)
+    np.testing.assert_allclose(l0, l8, rtol=0, atol=1e-12)   # the LSE does not depend on when m is raised
+    assert np.max(np.abs(l0 - lse)) < 0.5
+    with pytest.raises(ValueError):
+        oracle.fp8_attention_forward(q, k, v, False, scale, sigma, tau=1.0)   # 2 * 256 > 448
+
+
+def test_fp8_deferred_max_two_tile_closed_form():
+    """Two keys visited one per tile, log2-domain scores 0 and 0.5 (scale = ln 2,
+    so c = scale log2 e = 1; Q = e_0, K_1 = 0.5 e_0: every operand and block
+    scale exact in e4m3). With tau = 0.8 the second tile's max (0.5) does not
+    raise m = 0, so P~ = [1, 2^0.5] and, with w = 256 (one V block),
+    P~ w = [256, 362.04] -> e4m3 [256, 352] (quantum 32 in [256, 448): 11.31
+    quanta round to 11): O = (V_0 + 1.375 V_1) / (1 + 2^0.5). With tau = 0
+    the max is raised to 0.5 and every code is exact: O is the softmax's."""
+    q = np.zeros((1, 1, 2, 4))
+    q[..., 0] = 1.0
+    k = np.zeros((1, 1, 2, 4))
+    k[0, 0, 1, 0] = 0.5
+    v = np.zeros((1, 1, 2, 4))
+    v[0, 0, 0] = [2.0, -1.0, 0.5, 0.0]
+    v[0, 0, 1] = [1.0, 2.0, -2.0, 0.25]
+    scale = math.log(2.0)
+    # rtol 1e-6: V's block scale 2/448 is a float32 value (relative error
+    # below 2^-24); the two readings differ by 3 % (1.375 against 2^0.5)
+    o8, _ = oracle.fp8_attention_forward(q, k, v, False, scale, None, tile=1, tau=0.8)
+    want = (v[0, 0, 0] + 1.375 * v[0, 0, 1]) / (1 + 2 ** 0.5)
+    np.testing.assert_allclose(o8[0, 0, 0], want, rtol=1e-6, atol=1e-9)
+    o0, _ = oracle.fp8_attention_forward(q, k, v, False, scale, None, tile=1, tau=0.0)
+    exact = (2 ** -0.5 * v[0, 0, 0] + v[0, 0, 1]) / (1 + 2 ** -0.5)
+    np.testing.assert_allclose(o0[0, 0, 0], exact, rtol=1e-6, atol=1e-9)
