@@ -12,6 +12,9 @@ from .api import (  # noqa: F401
     fa_fwd,
     fa_bwd,
     fa_bwd_noalloc,
+    fa_fwd_varlen,
+    fa_bwd_varlen,
+    fa_bwd_varlen_workspace_size,
     fa_fwd_fp8,
     fa_fp8_quantize,
     fa_fwd_fp8_quantized,

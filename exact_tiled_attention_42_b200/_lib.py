@@ -30,6 +30,9 @@ SIGNATURES = {
     "fa_fp8_quantize": (_c_int, [_c_void_p] * 3 + [_c_uint64, _c_int, _c_void_p, _c_size_t] + [_c_int] * 5 + [_c_void_p]),
     "fa_fwd_fp8_quantized": (_c_int, [_c_void_p, _c_size_t, _c_void_p, _c_void_p] + [_c_int] * 7 + [_c_float, _c_void_p]),
     "fa_fwd_decode": (_c_int, [_c_void_p] * 6 + [_c_size_t] + [_c_int] * 7 + [_c_float, _c_int, _c_void_p]),
+    "fa_fwd_varlen": (_c_int, [_c_void_p] * 6 + [_c_int] * 7 + [_c_float, _c_void_p]),
+    "fa_bwd_varlen_workspace_size": (_c_size_t, [_c_int] * 6),
+    "fa_bwd_varlen": (_c_int, [_c_void_p] * 11 + [_c_size_t] + [_c_int] * 7 + [_c_float, _c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [_c_int]),
     "fa_last_device_status": (_c_int, []),
 }

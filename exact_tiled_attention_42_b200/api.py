@@ -233,3 +233,66 @@ def fa_fwd_decode(q, k, v, causal: bool = False, scale: float | None = None, num
     if st != FA_OK:
         raise FAError("fa_fwd_decode", st)
     return out, lse
+
+
+def _varlen_dims(q, k, cu_seqlens):
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("packed q and k must be [T, H, d]")
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if not isinstance(cu_seqlens, torch.Tensor) or not cu_seqlens.is_cuda or cu_seqlens.dtype != torch.int32 \
+            or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+        raise TypeError("cu_seqlens must be a contiguous int32 CUDA tensor of B + 1 offsets")
+    return cu_seqlens.numel() - 1, T, Hq, Hkv, d
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool = False, scale: float | None = None,
+                  out=None, lse=None, stream=None):
+    """Packed variable-length batch: q [T, Hq, d], k/v [T, Hkv, d] bf16,
+    sequence b = tokens cu_seqlens[b]..cu_seqlens[b+1]-1 (int32 CUDA tensor),
+    max_seqlen >= every length. Returns O [T, Hq, d] bf16, LSE [Hq, T] fp32."""
+    B, T, Hq, Hkv, d = _varlen_dims(q, k, cu_seqlens)
+    _check("q", q, torch.bfloat16, (T, Hq, d))
+    _check("k", k, torch.bfloat16, (T, Hkv, d))
+    _check("v", v, torch.bfloat16, (T, Hkv, d))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check("out", out, torch.bfloat16, (T, Hq, d))
+    _check("lse", lse, torch.float32, (Hq, T))
+    st = _lib.load().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                   cu_seqlens.data_ptr(), B, Hq, Hkv, T, int(max_seqlen), d, int(bool(causal)),
+                                   float(scale), _stream(stream))
+    if st != FA_OK:
+        raise FAError("fa_fwd_varlen", st)
+    return out, lse
+
+
+def fa_bwd_varlen_workspace_size(B: int, Hq: int, Hkv: int, total: int, max_seqlen: int, d: int) -> int:
+    return int(_lib.load().fa_bwd_varlen_workspace_size(B, Hq, Hkv, total, max_seqlen, d))
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens, max_seqlen: int, causal: bool = False,
+                  scale: float | None = None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of a packed variable-length batch (layouts of fa_fwd_varlen)."""
+    B, T, Hq, Hkv, d = _varlen_dims(q, k, cu_seqlens)
+    for name, t, shp in (("q", q, (T, Hq, d)), ("k", k, (T, Hkv, d)), ("v", v, (T, Hkv, d)),
+                         ("o", o, (T, Hq, d)), ("dout", dout, (T, Hq, d))):
+        _check(name, t, torch.bfloat16, shp)
+    _check("lse", lse, torch.float32, (Hq, T))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        n = fa_bwd_varlen_workspace_size(B, Hq, Hkv, T, int(max_seqlen), d)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    st = _lib.load().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu_seqlens.data_ptr(),
+                                   workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                   B, Hq, Hkv, T, int(max_seqlen), d, int(bool(causal)), float(scale), _stream(stream))
+    if st != FA_OK:
+        raise FAError("fa_bwd_varlen", st)
+    return dq, dk, dv

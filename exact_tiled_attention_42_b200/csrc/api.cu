@@ -51,11 +51,17 @@ int* status_ptr() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-fa_status check_shape(int B, int Hq, int Hkv, int N, int d, float scale) {
+#ifdef FA_DEBUG_WITHHOLD
+int g_debug_withhold = 0;  // debug build only: read by fa_fwd at each call
+#endif
+
+// Head dimensions: 64, 96 and 128 everywhere; 192 and 256 for the forward
+// entry points (wide = true).
+fa_status check_shape(int B, int Hq, int Hkv, int N, int d, float scale, bool wide = false) {
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return FA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 96 && d != 128 && !(wide && (d == 192 || d == 256))) return FA_ERR_UNSUPPORTED;
   // one 1-D grid of (batch x head) x (query or key tiles): must fit in 2^31 - 1
   const long long BH = static_cast<long long>(B) * Hq;
   const long long tiles = (N + 127) / 128;
@@ -77,6 +83,22 @@ bool make_map_bf16(CUtensorMap* m, const void* ptr, int d, int N, long long oute
   return r == CUDA_SUCCESS;
 }
 
+// 3-D map over a token-major packed [T, H, d] bf16 tensor: boxes of 64
+// columns x 1 head x 128 tokens (the same 128-row x 128-byte shared-memory
+// tile as make_map_bf16's).
+bool make_map_bf16_packed(CUtensorMap* m, const void* ptr, int d, long long H, long long T, int box_rows = 128) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 3-D map over the fp32 dQ accumulator [BH, N, d]: 16 x 32 boxes, 64B swizzle
 // (the layout the backward's drain warps stage rows in).
 bool make_map_f32_acc(CUtensorMap* m, const void* ptr, int d, int N, long long outer) {
@@ -85,6 +107,21 @@ bool make_map_f32_acc(CUtensorMap* m, const void* ptr, int d, int N, long long o
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(outer)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(N) * d * 4};
   cuuint32_t box[3] = {16, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3-D map over a packed fp32 dQ accumulator [T, Hq, d]: boxes of 16 columns
+// x 1 head x 32 tokens, 64B swizzle (the drain's staging layout).
+bool make_map_f32_acc_packed(CUtensorMap* m, const void* ptr, int d, long long H, long long T) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(H) * d * 4};
+  cuuint32_t box[3] = {16, 1, 32};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -139,6 +176,14 @@ const char* fa_status_string(fa_status s) {
   return "FA_ERR_UNKNOWN";
 }
 
+#ifdef FA_DEBUG_WITHHOLD
+// Debug build only (libfa_b200_debug.so, built with a 1 ms wait bound): while
+// `on` is non-zero, fa_fwd's producer never issues its first V tile, so a
+// bounded wait in every CTA runs out and reports FA_ERR_TIMEOUT. For the test
+// of the abort path; the release library has no such switch.
+void fa_debug_withhold_first_v(int on) { g_debug_withhold = on != 0; }
+#endif
+
 int fa_last_device_status(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return -1;
   int v = 0;
@@ -151,17 +196,22 @@ int fa_last_device_status(void) {
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
                  int d, int causal, float scale, cudaStream_t stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-  fa_status st = check_shape(B, Hq, Hkv, N, d, scale);
+  fa_status st = check_shape(B, Hq, Hkv, N, d, scale, true);
   if (st != FA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  const bool wide = d > 128;  // 64-key tiles for K and V
   CUtensorMap tmQ, tmK, tmV, tmO;
   const long long BH = static_cast<long long>(B) * Hq, BHkv = static_cast<long long>(B) * Hkv;
-  if (!make_map_bf16(&tmQ, q, d, N, BH, 128) || !make_map_bf16(&tmK, k, d, N, BHkv, 128) ||
-      !make_map_bf16(&tmV, v, d, N, BHkv, 128) || !make_map_bf16(&tmO, o, d, N, BH, 128))
+  if (!make_map_bf16(&tmQ, q, d, N, BH, 128) || !make_map_bf16(&tmK, k, d, N, BHkv, wide ? 64 : 128) ||
+      !make_map_bf16(&tmV, v, d, N, BHkv, wide ? 64 : 128) || !make_map_bf16(&tmO, o, d, N, BH, 128))
     return FA_ERR_CUDA;
   fa::FwdParams p;
   p.lse = lse;
   p.status = status_ptr();
+  p.cu_seqlens = nullptr;
+  p.o = static_cast<uint16_t*>(o);
+  p.total = 0;
+  p.d = d;
   p.N = N;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -169,8 +219,55 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.num_qtiles = (N + 127) / 128;
   p.num_pairs = (p.num_qtiles + 1) / 2;
   p.scale_log2 = scale * 1.4426950408889634f;
+#ifdef FA_DEBUG_WITHHOLD
+  p.debug_withhold = g_debug_withhold;
+#endif
   if (!p.status) return FA_ERR_CUDA;
-  cudaError_t e = fa::launch_fwd_bf16(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), d, causal != 0, stream);
+  cudaError_t e = wide ? fa::launch_fwd_wide(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), d, causal != 0, stream)
+                       : fa::launch_fwd_bf16(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), d, causal != 0, stream);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
+                        int B, int Hq, int Hkv, int total, int max_seqlen, int d, int causal, float scale,
+                        cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse || !cu_seqlens) return FA_ERR_INVALID_ARG;
+  if (total < 0 || max_seqlen < 0) return FA_ERR_INVALID_ARG;
+  if (total == 0 || max_seqlen == 0) {  // every sequence is empty: nothing to compute
+    fa_status st = check_shape(B, Hq, Hkv, 1, d, scale, true);
+    return st;
+  }
+  fa_status st = check_shape(B, Hq, Hkv, max_seqlen, d, scale, true);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+    return FA_ERR_MISALIGNED;
+  const bool wide = d > 128;
+  CUtensorMap tmQ, tmK, tmV, tmO;
+  if (!make_map_bf16_packed(&tmQ, q, d, Hq, total) || !make_map_bf16_packed(&tmK, k, d, Hkv, total, wide ? 64 : 128) ||
+      !make_map_bf16_packed(&tmV, v, d, Hkv, total, wide ? 64 : 128) || !make_map_bf16_packed(&tmO, o, d, Hq, total))
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.lse = lse;
+  p.status = status_ptr();
+  p.cu_seqlens = cu_seqlens;
+  p.o = static_cast<uint16_t*>(o);
+  p.total = total;
+  p.d = d;
+  p.N = max_seqlen;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.num_qtiles = (max_seqlen + 127) / 128;
+  p.num_pairs = (p.num_qtiles + 1) / 2;
+  p.scale_log2 = scale * 1.4426950408889634f;
+#ifdef FA_DEBUG_WITHHOLD
+  p.debug_withhold = 0;
+#endif
+  if (!p.status) return FA_ERR_CUDA;
+  const long long BH = static_cast<long long>(B) * Hq;
+  cudaError_t e = wide ? fa::launch_fwd_wide(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), d, causal != 0, stream)
+                       : fa::launch_fwd_bf16(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), d, causal != 0, stream);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -205,6 +302,10 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.neg_lse2 = reinterpret_cast<float*>(ws + vec_bytes);
   p.dq_accum = reinterpret_cast<float*>(ws + 2 * vec_bytes);
   p.dq = static_cast<uint16_t*>(dq);
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
+  p.cu_seqlens = nullptr;
+  p.total = 0;
   p.status = status_ptr();
   p.N = N;
   p.Npad = T * 128;
@@ -213,6 +314,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.group = Hq / Hkv;
   p.num_tiles = T;
   p.d = d;
+  p.d_pad = d == 64 ? 64 : 128;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   if (!p.status) return FA_ERR_CUDA;
@@ -221,6 +323,69 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
       !make_map_bf16(&tmV, v, d, N, BHkv, 128) || !make_map_bf16(&tmdO, dout, d, N, BH, 128) ||
       !make_map_bf16(&tmdK, dk, d, N, BHkv, 128) || !make_map_bf16(&tmdV, dv, d, N, BHkv, 128) ||
       !make_map_f32_acc(&tmAcc, p.dq_accum, d, N, BH))
+    return FA_ERR_CUDA;
+  cudaError_t e = fa::launch_bwd_bf16(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmAcc, p, B, causal != 0, stream);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_varlen_workspace_size(int B, int Hq, int Hkv, int total, int max_seqlen, int d) {
+  if (total < 0 || max_seqlen < 0 || check_shape(B, Hq, Hkv, max_seqlen > 0 ? max_seqlen : 1, d, 1.0f) != FA_OK)
+    return 0;
+  const size_t bh = static_cast<size_t>(B) * Hq;
+  const size_t npad = static_cast<size_t>((max_seqlen + 127) / 128) * 128;
+  const size_t ws = 2 * up256(bh * npad * sizeof(float)) + up256(static_cast<size_t>(total) * Hq * d * sizeof(float));
+  return ws > 0 ? ws : 256;
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, const int* cu_seqlens, void* workspace,
+                        size_t workspace_bytes, int B, int Hq, int Hkv, int total, int max_seqlen, int d, int causal,
+                        float scale, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !cu_seqlens) return FA_ERR_INVALID_ARG;
+  if (total < 0 || max_seqlen < 0) return FA_ERR_INVALID_ARG;
+  fa_status st = check_shape(B, Hq, Hkv, max_seqlen > 0 ? max_seqlen : 1, d, scale);
+  if (st != FA_OK) return st;
+  if (total == 0 || max_seqlen == 0) return FA_OK;  // every sequence is empty: nothing to compute
+  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < fa_bwd_varlen_workspace_size(B, Hq, Hkv, total, max_seqlen, d))
+    return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  const long long BH = static_cast<long long>(B) * Hq;
+  const int T = (max_seqlen + 127) / 128;
+  const size_t vec_bytes = up256(static_cast<size_t>(BH) * T * 128 * sizeof(float));
+  char* ws = static_cast<char*>(workspace);
+  fa::BwdParams p;
+  p.o = static_cast<const uint16_t*>(o);
+  p.dout = static_cast<const uint16_t*>(dout);
+  p.lse = lse;
+  p.delta = reinterpret_cast<float*>(ws);
+  p.neg_lse2 = reinterpret_cast<float*>(ws + vec_bytes);
+  p.dq_accum = reinterpret_cast<float*>(ws + 2 * vec_bytes);
+  p.dq = static_cast<uint16_t*>(dq);
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
+  p.cu_seqlens = cu_seqlens;
+  p.total = total;
+  p.status = status_ptr();
+  p.N = max_seqlen;
+  p.Npad = T * 128;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.num_tiles = T;
+  p.d = d;
+  p.d_pad = d == 64 ? 64 : 128;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (!p.status) return FA_ERR_CUDA;
+  CUtensorMap tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmAcc;
+  if (!make_map_bf16_packed(&tmQ, q, d, Hq, total) || !make_map_bf16_packed(&tmK, k, d, Hkv, total) ||
+      !make_map_bf16_packed(&tmV, v, d, Hkv, total) || !make_map_bf16_packed(&tmdO, dout, d, Hq, total) ||
+      !make_map_bf16_packed(&tmdK, dk, d, Hkv, total) || !make_map_bf16_packed(&tmdV, dv, d, Hkv, total) ||
+      !make_map_f32_acc_packed(&tmAcc, p.dq_accum, d, Hq, total))
     return FA_ERR_CUDA;
   cudaError_t e = fa::launch_bwd_bf16(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmAcc, p, B, causal != 0, stream);
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;

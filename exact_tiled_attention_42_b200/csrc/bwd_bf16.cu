@@ -21,6 +21,9 @@
 //   dV  += P^T dO_i       (P^T from tensor memory, bf16)
 //   dK  += dS^T Q_i       (dS^T from tensor memory, bf16)
 //   dQ_i = dS K_j         (dS from shared memory, MN-major)
+// issued in the order dP^T(i), dV(i), S^T(i+1), dK(i), dQ(i): the next S^T
+// starts as soon as dV has read P^T, so the compute warps form P^T(i+1) while
+// the tensor cores run dK(i) and dQ(i).
 // Roles, 512 threads in four warpgroups: warpgroups 0 and 1 turn S^T into P^T
 // and dP^T into dS^T (thread = key row; query columns [0,64) and [64,128), so
 // two warps per scheduler share the exponentials); warpgroup 2 drains dQ_i out
@@ -33,10 +36,12 @@
 // the drain to 152 -- 256 * 136 + 128 * 152 + 128 * 88 = 512 * 128, checked
 // against the compiled register count on the host before launching.
 // Each compute warpgroup writes its P^T (bf16) over the first 32 of its 64
-// S^T columns and its dS^T over the next 32; for d = 128 the dQ accumulator
-// reuses the dP^T columns and dS reuses the shared-memory slot of dO_i once dV
-// has read it. dK is issued as soon as dS^T is in tensor memory, before dS has
-// reached shared memory (which waits for dV), and dQ once it has.
+// S^T columns (and keeps it in registers for dS, since the next S^T lands in
+// those columns) and its dS^T over the first 32 of its 64 dP^T columns; for
+// d = 128 the dQ accumulator then reuses the dP^T columns, and dS reuses the
+// shared-memory slot of dO_i once dV has read it. dK is issued as soon as
+// dS^T is in tensor memory, before dS has reached shared memory (which waits
+// for dV), and dQ once it has.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -70,8 +75,8 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_VEC + 2048;
   static constexpr int NUM_BARS = 20;
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
-  static constexpr uint32_t COL_S = 0;    // S^T; then per 64 queries: P^T bf16 in +[0,32), dS^T in +[32,64)
-  static constexpr uint32_t COL_DP = 128;
+  static constexpr uint32_t COL_S = 0;    // S^T; then per 64 queries: P^T bf16 in +[0,32)
+  static constexpr uint32_t COL_DP = 128;  // dP^T; then per 64 queries: dS^T bf16 in +[0,32)
   static constexpr uint32_t COL_DV = 256;
   static constexpr uint32_t COL_DK = 256 + D;
   static constexpr uint32_t COL_DQ = (D == 64) ? 384 : 128;
@@ -115,17 +120,30 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 // up to Npad), and zeros in the fp32 dQ accumulator. d/8 lanes per row, each
 // covering 8 consecutive elements.
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p, long long total_rows) {
-  const int lpr = p.d >> 3;
+  const int lpr = p.d_pad >> 3;  // lanes per row (a power of two)
   const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long row = gt / lpr;
   const int sub = static_cast<int>(gt - row * lpr);
   const bool valid = row < total_rows;
   const long long bh = valid ? row / p.Npad : 0;
   const int n = valid ? static_cast<int>(row - bh * p.Npad) : 0;
-  const bool real = valid && n < p.N;
+  // the row's sequence: fixed length N, or a packed batch's sequence b
+  long long tok = 0;  // row index of [B*Hq, N] (fixed) or token index of [T, Hq] (packed)
+  int len = p.N;
+  if (p.cu_seqlens) {
+    const int b = static_cast<int>(bh / p.Hq);
+    const int s0 = p.cu_seqlens[b];
+    len = p.cu_seqlens[b + 1] - s0;
+    if (len < 0 || len > p.N || s0 < 0 || s0 + len > p.total) len = 0;  // reported by the main kernel
+    tok = (static_cast<long long>(s0) + n) * p.Hq + (bh - static_cast<long long>(b) * p.Hq);
+  } else {
+    tok = bh * p.N + n;
+  }
+  const bool real = valid && n < len;
+  const bool col = sub * 8 < p.d;
   float acc = 0.f;
-  if (real) {
-    const long long off = (bh * p.N + n) * p.d + sub * 8;
+  if (real && col) {
+    const long long off = tok * p.d + sub * 8;
     const uint4 ov = *reinterpret_cast<const uint4*>(p.o + off);
     const uint4 gv = *reinterpret_cast<const uint4*>(p.dout + off);
     const uint32_t oa[4] = {ov.x, ov.y, ov.z, ov.w};
@@ -139,7 +157,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p, long lo
   for (int off = lpr >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (valid && sub == 0) {
     p.delta[row] = real ? acc : 0.f;
-    p.neg_lse2[row] = real ? -p.lse[bh * p.N + n] * LOG2E : 0.f;
+    const long long lse_i = p.cu_seqlens ? (bh - (bh / p.Hq) * p.Hq) * p.total + (tok / p.Hq) : bh * p.N + n;
+    p.neg_lse2[row] = real ? -p.lse[lse_i] * LOG2E : 0.f;
   }
 }
 
@@ -173,7 +192,7 @@ struct QWalk {
   }
 };
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -194,10 +213,31 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const int j = static_cast<int>(blockIdx.x) - bkv * p.num_tiles;  // key tile
   const int b = bkv / p.Hkv;
   const int kvh = bkv - b * p.Hkv;
-  const int T = p.num_tiles;
+  // A packed batch's sequence b: tokens s0 .. s0 + len - 1. CTAs whose key
+  // tile lies past the sequence's end leave at once.
+  int s0 = 0, len = p.N;
+  if (VARLEN) {
+    s0 = p.cu_seqlens[b];
+    len = p.cu_seqlens[b + 1] - s0;
+    if (len < 0 || len > p.N || s0 < 0 || s0 + len > p.total) {
+      if (threadIdx.x == 0 && j == 0) report_status(p.status, FA_ERR_INVALID_ARG | (SITE_SEQLENS << 8));
+      return;
+    }
+  }
+  const int T = VARLEN ? (len + BT - 1) / BT : p.num_tiles;
+  if (VARLEN && j >= T) return;
   const int i0 = CAUSAL ? j : 0;
   const int nq = T - i0;
   const int n_it = p.group * nq;
+  // TMA coordinates of 128 rows starting at row r of a head (fixed: y = row,
+  // z = head; packed: y = head, z = token)
+  auto tma_rows = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int x, int r, int head) {
+    if (VARLEN)
+      tma_load_3d(dst, m, bar, x, head, s0 + r);
+    else
+      tma_load_3d(dst, m, bar, x, r, head);
+  };
+  const int kv_head = VARLEN ? kvh : bkv;  // K, V, dK, dV map head coordinate
 
   const BwdBars bars{base + C::OFF_BAR};
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_BAR + C::NUM_BARS * 8);
@@ -244,6 +284,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   // Iteration it visits query head (it / nq) of the group and query tile
   // i0 + it % nq. Each role walks these in order with a QWalk (no division).
   const int bhq0 = b * p.Hq + kvh * p.group;  // first query head of the group, as b * Hq + hq
+  const int qhead0 = VARLEN ? kvh * p.group : bhq0;  // its Q, dO, dQ map head coordinate
   auto ds_smem = [&](int st) -> uint32_t {
     return C::DS_ALIAS ? base + C::OFF_DO + st * C::TILE_BYTES : base + C::OFF_DS;
   };
@@ -256,8 +297,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (lane == 0) {
         mbar_arrive_expect_tx(bars.kv_full(), 2 * C::TILE_BYTES);
         for (int bx = 0; bx < C::BOXES; ++bx) {
-          tma_load_3d(base + C::OFF_K + bx * C::BOX_BYTES, &tmK, bars.kv_full(), bx * 64, j * BT, bkv);
-          tma_load_3d(base + C::OFF_V + bx * C::BOX_BYTES, &tmV, bars.kv_full(), bx * 64, j * BT, bkv);
+          tma_rows(base + C::OFF_K + bx * C::BOX_BYTES, &tmK, bars.kv_full(), bx * 64, j * BT, kv_head);
+          tma_rows(base + C::OFF_V + bx * C::BOX_BYTES, &tmV, bars.kv_full(), bx * 64, j * BT, kv_head);
         }
         int issued = 0;
         QWalk qw(i0, T);
@@ -265,12 +306,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           const int st = it & 1;
           const uint32_t ph = (it >> 1) & 1;
           const int bhq = bhq0 + qw.head;
+          const int qh = qhead0 + qw.head;
           const int i = qw.tile;
           if (!mbar_wait_sleep(bars.q_empty(st), ph ^ 1, abort, p.status, SITE_BWD + 1)) break;
           mbar_arrive_expect_tx(bars.q_full(st), C::TILE_BYTES + 1024);
           for (int bx = 0; bx < C::BOXES; ++bx)
-            tma_load_3d(base + C::OFF_Q + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, bars.q_full(st), bx * 64,
-                        i * BT, bhq);
+            tma_rows(base + C::OFF_Q + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, bars.q_full(st), bx * 64,
+                     i * BT, qh);
           const long long voff = static_cast<long long>(bhq) * p.Npad + i * BT;
           bulk_load_1d(base + C::OFF_VEC + st * 1024, p.neg_lse2 + voff, 512, bars.q_full(st));
           bulk_load_1d(base + C::OFF_VEC + st * 1024 + 512, p.delta + voff, 512, bars.q_full(st));
@@ -280,8 +322,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           }
           mbar_arrive_expect_tx(bars.do_full(st), C::TILE_BYTES);
           for (int bx = 0; bx < C::BOXES; ++bx)
-            tma_load_3d(base + C::OFF_DO + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmdO, bars.do_full(st), bx * 64,
-                        i * BT, bhq);
+            tma_rows(base + C::OFF_DO + st * C::TILE_BYTES + bx * C::BOX_BYTES, &tmdO, bars.do_full(st), bx * 64,
+                     i * BT, qh);
           issued = 2 * it + 2;
         }
         if (*abort) {
@@ -300,21 +342,31 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         constexpr uint32_t IDESC_TS = idesc_bf16(BT, D, false, true);
         constexpr uint32_t IDESC_DQ = idesc_bf16(BT, D, true, true);
         const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
-        bool ok = mbar_wait_sleep(bars.kv_full(), 0, abort, p.status, SITE_BWD + 3);
-        for (int it = 0; ok && it < n_it; ++it) {
-          const int st = it & 1;
-          const uint32_t ph = (it >> 1) & 1;
-          const uint32_t sQ = base + C::OFF_Q + st * C::TILE_BYTES;
-          const uint32_t sdO = base + C::OFF_DO + st * C::TILE_BYTES;
-          if (!mbar_wait_sleep(bars.q_full(st), ph, abort, p.status, SITE_BWD + 4)) break;
-          tc_fence_after();
+        auto issue_st = [&](int it) {  // S^T = K_j Q_i^T into the S^T columns
+          const uint32_t sQ = base + C::OFF_Q + (it & 1) * C::TILE_BYTES;
   #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K_j Q_i^T
+          for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
             mma_ss(tmem + C::COL_S, smem_desc_sw128(sK + off, 16, 1024), smem_desc_sw128(sQ + off, 16, 1024),
                    IDESC_SS, kk > 0 ? 1u : 0u);
           }
           mma_commit(bars.s_full());
+        };
+        bool ok = mbar_wait_sleep(bars.kv_full(), 0, abort, p.status, SITE_BWD + 3) &&
+                  mbar_wait_sleep(bars.q_full(0), 0, abort, p.status, SITE_BWD + 4);
+        if (ok) {
+          tc_fence_after();
+          issue_st(0);
+        }
+        // Per iteration: dP^T(it), dV(it), S^T(it + 1), dK(it), dQ(it). S^T(it + 1)
+        // goes into the S^T columns as soon as dV(it) has read P^T(it) from
+        // them (tcgen05 MMAs of one thread run in issue order), so the compute
+        // warps form P^T(it + 1) while the pipe runs dK(it) and dQ(it).
+        for (int it = 0; ok && it < n_it; ++it) {
+          const int st = it & 1;
+          const uint32_t ph = (it >> 1) & 1;
+          const uint32_t sQ = base + C::OFF_Q + st * C::TILE_BYTES;
+          const uint32_t sdO = base + C::OFF_DO + st * C::TILE_BYTES;
           if (!mbar_wait_sleep(bars.do_full(st), ph, abort, p.status, SITE_BWD + 5)) break;
           if (C::DQ_SHARES_DP && it > 0 && !mbar_wait_sleep(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
             break;
@@ -334,11 +386,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                    smem_desc_sw128(sdO + kk * 2048, C::BOX_BYTES, 1024),
                    IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bars.dv_done());
+          if (it + 1 < n_it) {
+            if (!mbar_wait_sleep(bars.q_full(st ^ 1), ((it + 1) >> 1) & 1, abort, p.status, SITE_BWD + 4)) break;
+            tc_fence_after();
+            issue_st(it + 1);
+          }
           if (!mbar_wait_sleep(bars.dst_ready(), it & 1, abort, p.status, SITE_BWD + 8)) break;
           tc_fence_after();
   #pragma unroll
-          for (int kk = 0; kk < BT / 16; ++kk)  // dK += dS^T Q_i
-            mma_ts(tmem + C::COL_DK, tmem + C::COL_S + (kk >> 2) * 64 + 32 + (kk & 3) * 8,
+          for (int kk = 0; kk < BT / 16; ++kk)  // dK += dS^T Q_i (dS^T over the dP^T columns)
+            mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + (kk >> 2) * 64 + (kk & 3) * 8,
                    smem_desc_sw128(sQ + kk * 2048, C::BOX_BYTES, 1024),
                    IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bars.q_empty(st));
@@ -366,8 +423,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::COL_S + 64 * half;  // S^T; then P^T at +0, dS^T at +32
-    const uint32_t tDP = tmem + lane_off + C::COL_DP + 64 * half;
+    const uint32_t tS = tmem + lane_off + C::COL_S + 64 * half;  // S^T; then P^T at +0
+    const uint32_t tDP = tmem + lane_off + C::COL_DP + 64 * half;  // dP^T; then dS^T at +0
     const float cl2 = p.scale_log2;
     bool ok = true;
     QWalk qw(i0, T);
@@ -382,7 +439,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const float* vec = reinterpret_cast<const float*>(base_ptr + C::OFF_VEC + st * 1024);
       const float* vec_lse = vec + 64 * half;
       const float* vec_d = vec + 128 + 64 * half;
-      const int qlim = p.N - i * BT - 64 * half;  // queries of this half past N are padding
+      const int qlim = len - i * BT - 64 * half;  // queries of this half past the end are padding
+      // a packed batch's keys past the sequence's end (the next sequence's
+      // tokens in the tile) take no part: P^T = 0 keeps them out of dS and dQ
+      const bool key_out = VARLEN && j * BT + r >= len;
+      uint32_t pk[32];  // P^T of this half, bf16 pairs: kept for dS
       {
         float s[64];
         {
@@ -413,7 +474,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           for (int c = 0; c < 64; ++c)
             if (c >= qlim) s[c] = 0.f;
         }
-        uint32_t pk[32];
+        if (key_out) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = 0.f;
+        }
 #pragma unroll
         for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(s[2 * e], s[2 * e + 1]);
         tmem_st_x16(tS, *reinterpret_cast<const uint32_t(*)[16]>(pk));
@@ -427,24 +491,27 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.dp_full(), it & 1, abort, p.status, SITE_BWD + 11));
       if (!ok) break;
       tc_fence_after();
-      // dS = P (dP - D), 32 queries at a time with P^T read back from tensor
-      // memory: into tensor memory first (dK can start at once), then into
-      // shared memory once dV has finished reading this dO slot (dQ)
+      // dS = P (dP - D), 32 queries at a time with P^T from registers (the S^T
+      // columns already hold the next S^T once dV has read P^T): into tensor
+      // memory over the first 32 of this warpgroup's 64 dP^T columns (each
+      // 16-column chunk is written only after the 32 columns it covers have
+      // been read), so dK can start at once, then into shared memory once dV
+      // has finished reading this dO slot (dQ)
       uint32_t dsk[32];
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        uint32_t t[32], pp[16];
+        uint32_t t[32];
         tmem_ld_x32(tDP + cc * 32, t);
-        tmem_ld_x16(tS + cc * 16, pp);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c = cc * 32 + 2 * e;
+          const uint32_t pp = pk[cc * 16 + e];
           const float2 dd = *reinterpret_cast<const float2*>(vec_d + c);
-          dsk[cc * 16 + e] = pack_bf16x2(bf16_lo(pp[e]) * (__uint_as_float(t[2 * e]) - dd.x),
-                                         bf16_hi(pp[e]) * (__uint_as_float(t[2 * e + 1]) - dd.y));
+          dsk[cc * 16 + e] = pack_bf16x2(bf16_lo(pp) * (__uint_as_float(t[2 * e]) - dd.x),
+                                         bf16_hi(pp) * (__uint_as_float(t[2 * e + 1]) - dd.y));
         }
-        tmem_st_x16(tS + 32 + cc * 16, *reinterpret_cast<const uint32_t(*)[16]>(dsk + cc * 16));
+        tmem_st_x16(tDP + cc * 16, *reinterpret_cast<const uint32_t(*)[16]>(dsk + cc * 16));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -469,10 +536,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     if (half != 0) ok = false;  // warpgroup 0 writes dK and dV
     if (ok) {
       tc_fence_after();
+      // A packed batch's last, partial key tile is written row by row: a
+      // tile-wide store would reach into the next sequence's rows.
+      const bool direct = VARLEN && (j + 1) * BT > len;
       for (int which = 0; which < 2; ++which) {
         const uint32_t src = tmem + lane_off + (which ? C::COL_DV : C::COL_DK);
         const float mul = which ? 1.0f : p.scale;
         const uint32_t stage = base + C::OFF_Q + which * C::TILE_BYTES;
+        uint16_t* const grow = (which ? p.dv : p.dk) + (static_cast<size_t>(s0 + j * BT + r) * p.Hkv + kvh) * p.d;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t t[32];
@@ -485,22 +556,34 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               w4[e] = pack_bf16x2(__uint_as_float(t[q * 8 + 2 * e]) * mul, __uint_as_float(t[q * 8 + 2 * e + 1]) * mul);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(box + sw128_offset(r, ((c & 63) >> 3) + q)),
-                         "r"(w4[0]), "r"(w4[1]), "r"(w4[2]), "r"(w4[3])
-                         : "memory");
+            if (direct) {
+              if (j * BT + r < len && c + q * 8 < p.d)
+                *reinterpret_cast<uint4*>(grow + c + q * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            } else {
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(box + sw128_offset(r, ((c & 63) >> 3) + q)),
+                           "r"(w4[0]), "r"(w4[1]), "r"(w4[2]), "r"(w4[3])
+                           : "memory");
+            }
           }
         }
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars.epi());
-      if (r == 0 && mbar_wait_sleep(bars.epi(), 0, abort, p.status, SITE_BWD + 14)) {
-        for (int bx = 0; bx < C::BOXES; ++bx) {
-          tma_store_3d(&tmdK, base + C::OFF_Q + bx * C::BOX_BYTES, bx * 64, j * BT, bkv);
-          tma_store_3d(&tmdV, base + C::OFF_Q + C::TILE_BYTES + bx * C::BOX_BYTES, bx * 64, j * BT, bkv);
+      if (!direct) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.epi());
+        if (r == 0 && mbar_wait_sleep(bars.epi(), 0, abort, p.status, SITE_BWD + 14)) {
+          for (int bx = 0; bx < C::BOXES; ++bx) {
+            if (VARLEN) {
+              tma_store_3d(&tmdK, base + C::OFF_Q + bx * C::BOX_BYTES, bx * 64, kvh, s0 + j * BT);
+              tma_store_3d(&tmdV, base + C::OFF_Q + C::TILE_BYTES + bx * C::BOX_BYTES, bx * 64, kvh, s0 + j * BT);
+            } else {
+              tma_store_3d(&tmdK, base + C::OFF_Q + bx * C::BOX_BYTES, bx * 64, j * BT, bkv);
+              tma_store_3d(&tmdV, base + C::OFF_Q + C::TILE_BYTES + bx * C::BOX_BYTES, bx * 64, j * BT, bkv);
+            }
+          }
+          bulk_commit();
+          bulk_wait_read0();
         }
-        bulk_commit();
-        bulk_wait_read0();
       }
     }
   } else {
@@ -514,7 +597,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     bool ok = true;
     QWalk qw(i0, T);
     for (int it = 0; ok && it < n_it; ++it) {
-      const int bhq = bhq0 + qw.head;
+      const int qh = qhead0 + qw.head;
       const int row0 = qw.tile * BT + w * 32;
       qw.next();
       ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.dq_full(), it & 1, abort, p.status, SITE_BWD + 15));
@@ -532,9 +615,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.dq_free());
-      if (row0 >= p.N) continue;  // every row of this warp is padding
+      if (row0 >= len) continue;  // every row of this warp is padding
+      // (rows of a partial tile past the end carry dQ = 0 exactly, since their
+      // P^T columns are 0: adding them into the next sequence's rows of a
+      // packed batch changes nothing)
 #pragma unroll
       for (int c16 = 0; c16 < D / 16; ++c16) {
+        if (c16 * 16 >= p.d) break;  // zero-padded columns (d = 96)
         const uint32_t buf = stg0 + (cnt & 1) * 2048;
         if (lane == 0) bulk_wait_read<1>();  // the reduce that last read this buffer is done with it
         __syncwarp();
@@ -548,7 +635,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_reduce_add_3d(&tmdQacc, buf, c16 * 16, row0, bhq);
+          if (VARLEN)
+            tma_reduce_add_3d(&tmdQacc, buf, c16 * 16, qh, s0 + row0);
+          else
+            tma_reduce_add_3d(&tmdQacc, buf, c16 * 16, row0, qh);
           bulk_commit();
         }
         ++cnt;
@@ -573,12 +663,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 cudaError_t launch_main(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                         const CUtensorMap& tmdO, const CUtensorMap& tmdK, const CUtensorMap& tmdV,
                         const CUtensorMap& tmdQacc, const BwdParams& p, int B, cudaStream_t stream) {
   using C = BwdCfg<D>;
-  auto kern = bwd_bf16_kernel<D, CAUSAL>;
+  auto kern = bwd_bf16_kernel<D, CAUSAL, VARLEN>;
   // the setmaxnreg increases wait until the CTA's register pool has room:
   // make sure the compiled launch allocation covers the split
   static int regs = 0;
@@ -596,6 +686,17 @@ cudaError_t launch_main(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CU
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_main_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                          const CUtensorMap& tmdO, const CUtensorMap& tmdK, const CUtensorMap& tmdV,
+                          const CUtensorMap& tmdQacc, const BwdParams& p, int B, bool causal, cudaStream_t stream) {
+  if (p.cu_seqlens)
+    return causal ? launch_main<D, true, true>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream)
+                  : launch_main<D, false, true>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream);
+  return causal ? launch_main<D, true, false>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream)
+                : launch_main<D, false, false>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_bwd_bf16(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
@@ -604,20 +705,21 @@ cudaError_t launch_bwd_bf16(const CUtensorMap& tmQ, const CUtensorMap& tmK, cons
                             cudaStream_t stream) {
   const long long BH = static_cast<long long>(B) * p.Hq;
   const long long rows = BH * p.Npad;
-  const long long threads = rows * (p.d / 8);
+  const long long threads = rows * (p.d_pad / 8);
   bwd_pre_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p, rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (p.d == 64)
-    e = causal ? launch_main<64, true>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream)
-               : launch_main<64, false>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream);
+  if (p.d_pad == 64)
+    e = launch_main_d<64>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, causal, stream);
   else
-    e = causal ? launch_main<128, true>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream)
-               : launch_main<128, false>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, stream);
+    e = launch_main_d<128>(tmQ, tmK, tmV, tmdO, tmdK, tmdV, tmdQacc, p, B, causal, stream);
   if (e != cudaSuccess) return e;
-  const long long n8 = BH * p.N * p.d / 8;
+  // dQ = scale * accumulator over every element of dQ's layout
+  const long long elems = p.cu_seqlens ? static_cast<long long>(p.total) * p.Hq * p.d : BH * p.N * p.d;
+  const long long n8 = elems / 8;
   long long blocks = (n8 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
   bwd_post_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p.dq_accum, p.dq, n8, p.scale);
   return cudaGetLastError();
 }

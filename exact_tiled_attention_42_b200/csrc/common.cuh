@@ -28,6 +28,7 @@ enum WaitSite : int {
   SITE_Q_FULL = 1, SITE_K_FULL, SITE_V_FULL, SITE_K_EMPTY, SITE_V_EMPTY,
   SITE_S_FULL, SITE_P_FULL, SITE_O_DONE, SITE_TEARDOWN, SITE_LOAD_DRAIN,
   SITE_BWD = 32,
+  SITE_SEQLENS = 64,  // a packed batch's offsets, checked on the device (FA_ERR_INVALID_ARG)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -304,6 +305,32 @@ __device__ __forceinline__ float exp2_poly(float x) {
   const float p = fmaf(fmaf(fmaf(C3, f, C2), f, C1), f, C0);
   const uint32_t j = static_cast<uint32_t>(__float_as_int(t) - __float_as_int(SHIFT));
   return __uint_as_float(__float_as_uint(p) + (j << 23));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Maximum of s[0 .. N), N a multiple of 8 and at least 24: eight independent
+// chains of three-input max over 8-column chunks, then the eight combined.
+template <int N>
+__device__ __forceinline__ float row_max(const float* s) {
+  static_assert(N % 8 == 0 && N >= 24, "row_max: N must be a multiple of 8, at least 24");
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = fmax3(s[i], s[i + 8], s[i + 16]);
+  constexpr int PAIRS = (N - 24) / 16;  // chunk pairs after the first three chunks
+#pragma unroll
+  for (int k = 0; k < PAIRS; ++k)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[24 + 16 * k + i], s[32 + 16 * k + i]);
+  if constexpr ((N - 24) % 16 != 0) {  // one chunk left
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[N - 8 + i]);
+  }
+  return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -100,7 +100,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -121,13 +121,36 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
   const int b = bh / p.Hq;
   const int hq = bh - b * p.Hq;
-  const int kvh = b * p.Hkv + hq / p.group;
+  // A packed batch's sequence b: tokens s0 .. s0 + len - 1 (its own N). CTAs
+  // whose query tiles lie past the sequence's end leave at once.
+  int s0 = 0, len = p.N;
+  if (VARLEN) {
+    s0 = p.cu_seqlens[b];
+    len = p.cu_seqlens[b + 1] - s0;
+    if (len < 0 || len > p.N || s0 < 0 || s0 + len > p.total) {
+      if (threadIdx.x == 0 && pair == 0) report_status(p.status, FA_ERR_INVALID_ARG | (SITE_SEQLENS << 8));
+      return;
+    }
+  }
+  const int num_qtiles = VARLEN ? (len + BM - 1) / BM : p.num_qtiles;
   const int qt0 = 2 * pair;
   const int qt1 = 2 * pair + 1;
-  const bool has1 = qt1 < p.num_qtiles;
-  const int n0 = CAUSAL ? qt0 + 1 : p.num_qtiles;
-  const int n1 = has1 ? (CAUSAL ? qt1 + 1 : p.num_qtiles) : 0;
+  if (VARLEN && qt0 >= num_qtiles) return;
+  // head coordinates of the TMA maps: [B*H, N, d] (fixed) or [T, H, d] (packed)
+  const int qhead = VARLEN ? hq : bh;
+  const int kvh = VARLEN ? hq / p.group : b * p.Hkv + hq / p.group;
+  const bool has1 = qt1 < num_qtiles;
+  const int n0 = CAUSAL ? qt0 + 1 : num_qtiles;
+  const int n1 = has1 ? (CAUSAL ? qt1 + 1 : num_qtiles) : 0;
   const int nkv = n0 > n1 ? n0 : n1;
+  // TMA coordinates of 128 rows starting at row r of a head (fixed: y = row,
+  // z = head; packed: y = head, z = token)
+  auto tma_rows = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar, int x, int r, int head) {
+    if (VARLEN)
+      tma_load_3d(dst, m, bar, x, head, s0 + r);
+    else
+      tma_load_3d(dst, m, bar, x, r, head);
+  };
 
   const Bars bars{base + C::OFF_BAR, C::NS};
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_BAR + C::NUM_BARS * 8);
@@ -174,10 +197,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         const uint32_t sQ = base + C::OFF_Q;
         mbar_arrive_expect_tx(bars.q_full(), (has1 ? 2 : 1) * C::TILE_BYTES);
         for (int bx = 0; bx < C::BOXES; ++bx)
-          tma_load_3d(sQ + bx * C::BOX_BYTES, &tmQ, bars.q_full(), bx * 64, qt0 * BM, bh);
+          tma_rows(sQ + bx * C::BOX_BYTES, &tmQ, bars.q_full(), bx * 64, qt0 * BM, qhead);
         if (has1)
           for (int bx = 0; bx < C::BOXES; ++bx)
-            tma_load_3d(sQ + C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, bars.q_full(), bx * 64, qt1 * BM, bh);
+            tma_rows(sQ + C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ, bars.q_full(), bx * 64, qt1 * BM, qhead);
         int issued = 0;
         for (int j = 0; j < nkv; ++j) {
           const int s = j % C::NS;
@@ -186,21 +209,32 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           mbar_arrive_expect_tx(bars.k_full(s), C::TILE_BYTES);
           const uint32_t sK = base + C::OFF_K + s * C::TILE_BYTES;
           for (int bx = 0; bx < C::BOXES; ++bx)
-            tma_load_3d(sK + bx * C::BOX_BYTES, &tmK, bars.k_full(s), bx * 64, j * BN, kvh);
+            tma_rows(sK + bx * C::BOX_BYTES, &tmK, bars.k_full(s), bx * 64, j * BN, kvh);
           if (!mbar_wait_sleep(bars.v_empty(s), ph ^ 1, abort, p.status, SITE_V_EMPTY)) {
             issued = 2 * j + 1;
             break;
           }
+#ifdef FA_DEBUG_WITHHOLD
+          // Debug build only: leave the first V tile out, so that the MMA
+          // warp's bounded wait for it runs out (the test of the abort path).
+          if (p.debug_withhold && j == 0) {
+            issued = 2 * j + 2;
+            continue;
+          }
+#endif
           mbar_arrive_expect_tx(bars.v_full(s), C::TILE_BYTES);
           const uint32_t sV = base + C::OFF_V + s * C::TILE_BYTES;
           for (int bx = 0; bx < C::BOXES; ++bx)
-            tma_load_3d(sV + bx * C::BOX_BYTES, &tmV, bars.v_full(s), bx * 64, j * BN, kvh);
+            tma_rows(sV + bx * C::BOX_BYTES, &tmV, bars.v_full(s), bx * 64, j * BN, kvh);
           issued = 2 * j + 2;
         }
         if (*abort) {
           // Let every copy already issued land before the CTA can exit.
           drain_wait(bars.q_full(), 0);
           for (int t = (issued > 2 * C::NS ? issued - 2 * C::NS : 0); t < issued; ++t) {
+#ifdef FA_DEBUG_WITHHOLD
+            if (p.debug_withhold && t == 1) continue;  // the V tile that was never issued
+#endif
             const int j = t >> 1;
             const uint32_t bar = (t & 1) ? bars.v_full(j % C::NS) : bars.k_full(j % C::NS);
             drain_wait(bar, (j / C::NS) & 1);
@@ -313,20 +347,14 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[c][i]);
       }
       const int kv0 = j * BN;
-      const bool edge = (kv0 + BN > p.N) || (CAUSAL && kv0 + BN - 1 > qt * BM);
+      const bool edge = (kv0 + BN > len) || (CAUSAL && kv0 + BN - 1 > qt * BM);
       if (edge) {
-        const int lim = CAUSAL ? min(qrow + 1, p.N) : p.N;  // keys [0, lim) are visible
+        const int lim = CAUSAL ? min(qrow + 1, len) : len;  // keys [0, lim) are visible
 #pragma unroll
         for (int c = 0; c < BN; ++c)
           if (kv0 + c >= lim) s[c] = -INFINITY;
       }
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = s[i];
-#pragma unroll
-      for (int c = 8; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-      const float tile_max = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * cl2;
+      const float tile_max = row_max<BN>(s) * cl2;
       if (j == 0) {
         m = tile_max;
       } else if (__any_sync(0xffffffffu, tile_max > m + TAU)) {
@@ -344,21 +372,23 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           tmem_st_x16(tO + c, r);
         }
       }
+      // P = 2^(c s - m), two scores per packed FMA and add
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(neg_m, neg_m);
+      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int qd = 0; qd < 4; ++qd) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float a = ex2(fmaf(s[qd * 32 + 2 * i], cl2, neg_m));
-          const float bb = ex2(fmaf(s[qd * 32 + 2 * i + 1], cl2, neg_m));
-          ls[i & 3] += a + bb;
-          pk[i] = pack_bf16x2(a, bb);
+          const float2 xx = __ffma2_rn(make_float2(s[qd * 32 + 2 * i], s[qd * 32 + 2 * i + 1]), c2, nm2);
+          const float2 ab = make_float2(ex2(xx.x), ex2(xx.y));
+          ls[i & 1] = __fadd2_rn(ls[i & 1], ab);
+          pk[i] = pack_bf16x2(ab.x, ab.y);
         }
         tmem_st_x16(tS + qd * 16, pk);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -369,6 +399,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       tc_fence_after();
       const float inv_l = 1.0f / l;
       const uint32_t stage = base + C::OFF_Q + x * C::TILE_BYTES;  // Q_x is no longer read
+      // A packed batch's last, partial query tile is written row by row: a
+      // tile-wide store would reach into the next sequence's rows.
+      const bool direct = VARLEN && (qt + 1) * BM > len;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t r[32];
@@ -381,23 +414,41 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             w[e] = pack_bf16x2(__uint_as_float(r[q * 8 + 2 * e]) * inv_l, __uint_as_float(r[q * 8 + 2 * e + 1]) * inv_l);
-          const uint32_t chunk = ((c & 63) >> 3) + q;
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(box + sw128_offset(row, chunk)), "r"(w[0]),
-                       "r"(w[1]), "r"(w[2]), "r"(w[3])
-                       : "memory");
+          if (direct) {
+            if (qrow < len && c + q * 8 < p.d)
+              *reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(s0 + qrow) * p.Hq + hq) * p.d + c + q * 8) =
+                  make_uint4(w[0], w[1], w[2], w[3]);
+          } else {
+            const uint32_t chunk = ((c & 63) >> 3) + q;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(box + sw128_offset(row, chunk)), "r"(w[0]),
+                         "r"(w[1]), "r"(w[2]), "r"(w[3])
+                         : "memory");
+          }
         }
       }
-      // Staged rows -> async proxy, then one thread stores the tile with TMA
-      // (rows at or past N are clipped by the tensor map).
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars.epi(x));
-      if (row == 0 && mbar_wait_sleep(bars.epi(x), 0, abort, p.status, SITE_O_DONE)) {
-        for (int bx = 0; bx < C::BOXES; ++bx) tma_store_3d(&tmO, stage + bx * C::BOX_BYTES, bx * 64, qt * BM, bh);
-        bulk_commit();
-        bulk_wait_read0();
+      if (!direct) {
+        // Staged rows -> async proxy, then one thread stores the tile with
+        // TMA (rows at or past N and columns past d are clipped by the map).
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.epi(x));
+        if (row == 0 && mbar_wait_sleep(bars.epi(x), 0, abort, p.status, SITE_O_DONE)) {
+          for (int bx = 0; bx < C::BOXES; ++bx) {
+            if (VARLEN)
+              tma_store_3d(&tmO, stage + bx * C::BOX_BYTES, bx * 64, hq, s0 + qt * BM);
+            else
+              tma_store_3d(&tmO, stage + bx * C::BOX_BYTES, bx * 64, qt * BM, bh);
+          }
+          bulk_commit();
+          bulk_wait_read0();
+        }
       }
-      if (qrow < p.N) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(l)) * LN2;
+      if (qrow < len) {
+        if (VARLEN)
+          p.lse[static_cast<size_t>(hq) * p.total + s0 + qrow] = (m + __log2f(l)) * LN2;
+        else
+          p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(l)) * LN2;
+      }
     }
   }
 
@@ -417,11 +468,11 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool VARLEN>
 cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
                    const FwdParams& p, int BH, cudaStream_t stream) {
   using C = FwdCfg<D>;
-  auto kern = fwd_bf16_kernel<D, CAUSAL>;
+  auto kern = fwd_bf16_kernel<D, CAUSAL, VARLEN>;
   // The softmax warpgroups' setmaxnreg.inc waits until the CTA's register
   // pool has room; make sure the compiled launch allocation covers the split.
   static int regs = 0;
@@ -439,15 +490,23 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
+                     const FwdParams& p, int BH, bool causal, cudaStream_t stream) {
+  if (p.cu_seqlens)
+    return causal ? launch<D, true, true>(tmQ, tmK, tmV, tmO, p, BH, stream)
+                  : launch<D, false, true>(tmQ, tmK, tmV, tmO, p, BH, stream);
+  return causal ? launch<D, true, false>(tmQ, tmK, tmV, tmO, p, BH, stream)
+                : launch<D, false, false>(tmQ, tmK, tmV, tmO, p, BH, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_fwd_bf16(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const CUtensorMap& tmO, const FwdParams& p, int BH, int d, bool causal,
                             cudaStream_t stream) {
-  if (d == 64) return causal ? launch<64, true>(tmQ, tmK, tmV, tmO, p, BH, stream)
-                             : launch<64, false>(tmQ, tmK, tmV, tmO, p, BH, stream);
-  return causal ? launch<128, true>(tmQ, tmK, tmV, tmO, p, BH, stream)
-                : launch<128, false>(tmQ, tmK, tmV, tmO, p, BH, stream);
+  if (d == 64) return launch_d<64>(tmQ, tmK, tmV, tmO, p, BH, causal, stream);
+  return launch_d<128>(tmQ, tmK, tmV, tmO, p, BH, causal, stream);  // d = 96 or 128
 }
 
 }  // namespace fa

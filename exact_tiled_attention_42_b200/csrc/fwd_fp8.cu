@@ -7,8 +7,8 @@
 // Asynchrony and Low-precision" (abstract) describes FP8 with block
 // quantisation; the forms used here:
 //   S = sQ(row block) sK(key block) (Qc Kc^T) scale / d       (kind::f8f6f4)
-//   running max and sum as in the bf16 path, but the max is raised on every
-//   increase so P <= 1;
+//   running max and sum as in the bf16 path, but a row raises its max once a
+//   tile's max exceeds it by more than TAU = 0.8 (not 8), so P <= 2^0.8;
 //   P~ = e4m3(P * sV(key block) / max sV * 256)               (V's block scale
 //        folded into P so that one MMA sums over key blocks with different
 //        scales; the 256 keeps small probabilities above e4m3's subnormals)
@@ -38,6 +38,19 @@ constexpr int REGS_OTHER = 88;
 static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * 168, "register split");
 constexpr float LN2 = 0.69314718055994530942f;
 constexpr float P_LIFT = 256.f;
+// A row raises its running max only when a tile's max exceeds it by more than
+// TAU (log2 units): P then stays below 2^TAU and P w below 2^TAU * 256 =
+// 445.7, inside e4m3's range.
+constexpr float TAU = 0.8f;
+static_assert(P_LIFT * 1.7411011f <= 448.f, "2^TAU * P_LIFT must stay within e4m3's range");
+// Of every 8 groups of 4 scores, this many take their exponentials on the FMA
+// pipe (exp2_poly) instead of MUFU.
+constexpr int POLY_GROUPS = 0;
+
+// exp2_poly on two values with packed FMA-pipe arithmetic.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  return make_float2(exp2_poly(x.x), exp2_poly(x.y));
+}
 
 struct Cfg {
   static constexpr int TILE_BYTES = BM * D;  // e4m3: 128 rows x 128 bytes
@@ -310,49 +323,61 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < BN; ++c)
           if (kv0 + c >= lim) s[c] = -INFINITY;
       }
-      float mx[8], mlo, mhi;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-      mlo = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-#pragma unroll
-      for (int c = 64; c < BN; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-      mhi = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      // row maxima of the two key halves (three-input max)
+      const float mlo = row_max<64>(s);
+      const float mhi = row_max<64>(s + 64);
       const float tile_max = fmaxf(mlo * f0, mhi * f1);
       if (j == 0) {
         m = tile_max;
-      } else if (__any_sync(0xffffffffu, tile_max > m)) {
-        const float m_new = fmaxf(m, tile_max);
-        const float alpha = ex2(m - m_new);
-        l *= alpha;
-        m = m_new;
+      } else {
+        // a row raises its max only past TAU; the warp rescales O in tensor
+        // memory when any of its rows did (alpha = 1 for the others)
+        const bool raise = tile_max > m + TAU;
+        if (__any_sync(0xffffffffu, raise)) {
+          const float m_new = raise ? fmaxf(m, tile_max) : m;
+          const float alpha = ex2(m - m_new);
+          l *= alpha;
+          m = m_new;
 #pragma unroll
-        for (int c = 0; c < D; c += 16) {
-          uint32_t r[16];
-          tmem_ld_x16(tO + c, r);
-          tmem_wait_ld();
+          for (int c = 0; c < D; c += 16) {
+            uint32_t r[16];
+            tmem_ld_x16(tO + c, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st_x16(tO + c, r);
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st_x16(tO + c, r);
+          }
         }
       }
-      const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      // P~ = 2^(c s - m), two scores per packed FMA; then P~ w with one
+      // packed multiply. (Folding log2 w into the exponent would save the
+      // multiply, but P~ = 1 for a row's largest key, and 2^(log2 w) is not
+      // exactly w: where w sits on an e4m3 rounding tie -- block scales are
+      // ratios of short bf16 values, so it can -- the code would flip.)
+      const float nm = (m == -INFINITY) ? 0.f : -m;
+      const float2 f0v = make_float2(f0, f0), f1v = make_float2(f1, f1), nmv = make_float2(nm, nm);
+      const float2 w0v = make_float2(w0, w0), w1v = make_float2(w1, w1);
+      float2 lsum[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float w = i < 16 ? w0 : w1;
-        const float f = i < 16 ? f0 : f1;
-        const float a0 = ex2(fmaf(s[4 * i], f, neg_m)), a1 = ex2(fmaf(s[4 * i + 1], f, neg_m));
-        const float a2 = ex2(fmaf(s[4 * i + 2], f, neg_m)), a3 = ex2(fmaf(s[4 * i + 3], f, neg_m));
-        ls[i & 3] += (a0 + a1) + (a2 + a3);
-        pk[i] = e4m3x4(a0 * w, a1 * w, a2 * w, a3 * w);
+        const bool hi = i >= 16;
+        const float2 x01 = __ffma2_rn(make_float2(s[4 * i], s[4 * i + 1]), hi ? f1v : f0v, nmv);
+        const float2 x23 = __ffma2_rn(make_float2(s[4 * i + 2], s[4 * i + 3]), hi ? f1v : f0v, nmv);
+        float2 a01, a23;
+        if ((i & 7) < POLY_GROUPS) {
+          a01 = exp2_poly2(x01);
+          a23 = exp2_poly2(x23);
+        } else {
+          a01 = make_float2(ex2(x01.x), ex2(x01.y));
+          a23 = make_float2(ex2(x23.x), ex2(x23.y));
+        }
+        lsum[i & 1] = __fadd2_rn(lsum[i & 1], __fadd2_rn(a01, a23));
+        const float2 q01 = __fmul2_rn(a01, hi ? w1v : w0v), q23 = __fmul2_rn(a23, hi ? w1v : w0v);
+        pk[i] = e4m3x4(q01.x, q01.y, q23.x, q23.y);
       }
       tmem_st_x32(tS, pk);
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l += (lsum[0].x + lsum[0].y) + (lsum[1].x + lsum[1].y);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();

@@ -8,8 +8,18 @@
 namespace fa {
 
 struct FwdParams {
-  float* lse;        // [B*Hq, N]
+  float* lse;        // [B*Hq, N]; packed batches: [Hq, T]
   int* status;       // device status word (bounded waits report here)
+#ifdef FA_DEBUG_WITHHOLD
+  int debug_withhold;  // debug build only: 1 = the producer never issues the first V tile
+#endif
+  // Packed variable-length batches only (null otherwise): sequence b owns
+  // tokens cu_seqlens[b] .. cu_seqlens[b+1]-1 of the token-major [T, H, d]
+  // tensors, and N is the largest sequence length the grid was sized for.
+  const int* cu_seqlens;
+  uint16_t* o;       // packed batches: O [T, Hq, d] for the per-thread stores of partial tiles
+  int total;         // packed batches: T
+  int d;             // head dimension of the tensors (96 runs on the 128-column tiles, zero-padded)
   int N;
   int Hq;
   int Hkv;
@@ -20,27 +30,43 @@ struct FwdParams {
 };
 
 // tmQ/tmO: bf16 [B*Hq, N, d]; tmK/tmV: bf16 [B*Hkv, N, d]; all with
-// 64-column x 128-row boxes and 128-byte swizzle.
+// 64-column x 128-row boxes and 128-byte swizzle. Packed batches
+// (p.cu_seqlens set): tmQ/tmO over [T, Hq, d], tmK/tmV over [T, Hkv, d]
+// with 64-column x 1-head x 128-token boxes. d = 96 uses the d = 128 kernel:
+// the maps' inner extent is 96, so loads fill columns 96..127 with zeros and
+// stores clip them.
 cudaError_t launch_fwd_bf16(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const CUtensorMap& tmO, const FwdParams& p, int BH, int d, bool causal,
                             cudaStream_t stream);
 
+// Wide heads (d = 192, 256): one 128-row query tile per CTA and 64-key tiles
+// (grid BH * p.num_qtiles). tmQ/tmO as for launch_fwd_bf16; tmK/tmV with
+// 64-column x 64-row (packed: 64-token) boxes.
+cudaError_t launch_fwd_wide(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                            const CUtensorMap& tmO, const FwdParams& p, int BH, int d, bool causal,
+                            cudaStream_t stream);
+
 struct BwdParams {
-  const uint16_t* o;     // bf16 [B*Hq, N, d]   (preprocess)
-  const uint16_t* dout;  // bf16 [B*Hq, N, d]   (preprocess)
-  const float* lse;      // [B*Hq, N], natural log (preprocess)
-  float* delta;          // workspace [B*Hq, Npad]: D = rowsum(dO * O), 0 past N
-  float* neg_lse2;       // workspace [B*Hq, Npad]: -LSE * log2(e), 0 past N
-  float* dq_accum;       // workspace [B*Hq, N, d] fp32, zeroed by the preprocess
-  uint16_t* dq;          // bf16 [B*Hq, N, d]   (postprocess)
+  const uint16_t* o;     // bf16 [B*Hq, N, d] (packed batches: [T, Hq, d])  (preprocess)
+  const uint16_t* dout;  // bf16, as o                                      (preprocess)
+  const float* lse;      // [B*Hq, N] (packed: [Hq, T]), natural log        (preprocess)
+  float* delta;          // workspace [B*Hq, Npad]: D = rowsum(dO * O), 0 past each sequence's end
+  float* neg_lse2;       // workspace [B*Hq, Npad]: -LSE * log2(e), 0 past each sequence's end
+  float* dq_accum;       // workspace fp32, dQ's layout, zeroed by the preprocess
+  uint16_t* dq;          // bf16, dQ's layout                               (postprocess)
+  uint16_t* dk;          // packed batches: dK [T, Hkv, d] for the per-thread stores of partial tiles
+  uint16_t* dv;          // packed batches: dV, as dk
+  const int* cu_seqlens; // packed batches only (null otherwise): sequence offsets, B + 1 entries
   int* status;
-  int N;
-  int Npad;              // num_qtiles * 128
+  int total;             // packed batches: T
+  int N;                 // sequence length (packed batches: the largest)
+  int Npad;              // num_tiles * 128
   int Hq;
   int Hkv;
   int group;
   int num_tiles;         // ceil(N / 128): query tiles and key tiles
-  int d;
+  int d;                 // head dimension of the tensors
+  int d_pad;             // columns the kernel computes: 64 or 128 (d = 96 is zero-padded to 128)
   float scale;
   float scale_log2;
 };
@@ -48,7 +74,9 @@ struct BwdParams {
 // Backward: preprocess (D, -LSE*log2 e, zero dq_accum), the main kernel over
 // (key tile, KV head), and the dq postprocess. tmQ/tmdO: [B*Hq, N, d] bf16;
 // tmK/tmV/tmdK/tmdV: [B*Hkv, N, d] bf16 (64 x 128 boxes, 128B swizzle);
-// tmdQacc: fp32 [B*Hq, N, d] with 16 x 32 boxes and 64B swizzle.
+// tmdQacc: fp32 [B*Hq, N, d] with 16 x 32 boxes and 64B swizzle. Packed
+// batches (p.cu_seqlens set): the maps are over the token-major [T, H, d]
+// tensors with 1-head boxes of the same shapes.
 cudaError_t launch_bwd_bf16(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                             const CUtensorMap& tmdO, const CUtensorMap& tmdK, const CUtensorMap& tmdV,
                             const CUtensorMap& tmdQacc, const BwdParams& p, int B, bool causal,

@@ -24,7 +24,9 @@
  *   - Tensors are row-major contiguous: Q, O, dO, dQ are [B, Hq, N, d];
  *     K, V, dK, dV are [B, Hkv, N, d]; LSE and D are [B, Hq, N] float32.
  *     bf16 tensors are passed as raw 16-bit storage.
- *   - d is 64 or 128; N >= 1; Hq is a multiple of Hkv; scale is finite and > 0.
+ *   - d is 64, 96 or 128 (96 runs on the 128-column tiles with the extra
+ *     columns zero-filled on load and clipped on store; its FLOP cost is
+ *     that of 128); N >= 1; Hq is a multiple of Hkv; scale is finite and > 0.
  *   - Calls are asynchronous on `stream` (0 = legacy default stream), like a
  *     kernel launch; outputs are valid once the stream has been synchronised.
  *   - The caller owns every buffer, workspaces included. The library allocates
@@ -50,7 +52,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, Hq % Hkv != 0, bad scale */
-  FA_ERR_UNSUPPORTED = 2,  /* head dimension other than 64 / 128, or a size past the limits */
+  FA_ERR_UNSUPPORTED = 2,  /* head dimension not built for this entry point, or a size past the limits */
   FA_ERR_MISALIGNED = 3,   /* a pointer that is not 16-byte aligned */
   FA_ERR_WORKSPACE = 4,    /* workspace pointer null or smaller than the *_workspace_size query */
   FA_ERR_CUDA = 5,         /* the CUDA runtime reported an error when launching */
@@ -85,6 +87,50 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* workspace, size_t workspace_bytes,
                  int B, int Hq, int Hkv, int N, int d, int causal, float scale,
                  cudaStream_t stream);
+
+/*
+ * Packed variable-length batches. The blog page ("FlashAttention: The
+ * Algorithm That Made Long-Context AI Possible", section "Version 2 in 2023
+ * and version 3 in 2024") notes the method's uptake by training and serving
+ * stacks, whose batches pack sequences of different lengths end to end; the
+ * pages give no interface. Here every sequence is its own attention problem,
+ * exactly as if run alone:
+ *   - q, o, dq, dout: [T, Hq, d] bf16 and k, v, dk, dv: [T, Hkv, d] bf16,
+ *     token-major, T = total tokens; lse: [Hq, T] float32 (natural log).
+ *   - cu_seqlens: DEVICE pointer to B + 1 int32 offsets (4-byte aligned),
+ *     cu_seqlens[0] = 0, cu_seqlens[B] = T, non-decreasing; sequence b owns
+ *     tokens cu_seqlens[b] .. cu_seqlens[b+1] - 1 and may be empty.
+ *   - max_seqlen >= every sequence's length (the grid is sized by it).
+ *   - causal keeps key j for query i iff j <= i, positions local to the
+ *     sequence; nothing crosses a sequence boundary. GQA as in fa_fwd.
+ * The offsets are read on the device, so the host cannot check them: a
+ * sequence longer than max_seqlen or offsets outside [0, T] make the kernels
+ * skip that sequence and record FA_ERR_INVALID_ARG | (64 << 8) in the device
+ * status word (fa_last_device_status). T = 0 or max_seqlen = 0 returns FA_OK
+ * without launching. d is 64, 96 or 128.
+ */
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
+                        int B, int Hq, int Hkv, int total, int max_seqlen, int d, int causal, float scale,
+                        cudaStream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd_varlen needs: D and -LSE log2 e as float32
+ * [B * Hq, 128 * ceil(max_seqlen / 128)] and the float32 dQ accumulator
+ * [T, Hq, d], each rounded up to 256 bytes. Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_varlen_workspace_size(int B, int Hq, int Hkv, int total, int max_seqlen, int d);
+
+/*
+ * Backward of a packed variable-length batch by recomputation (fa_bwd's
+ * method, layouts and conventions of fa_fwd_varlen). `o` and `lse` are
+ * fa_fwd_varlen's outputs for the same inputs; dq, dk, dv are overwritten.
+ * The workspace is overwritten; its contents on entry do not matter.
+ */
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, const int* cu_seqlens,
+                        void* workspace, size_t workspace_bytes,
+                        int B, int Hq, int Hkv, int total, int max_seqlen, int d, int causal, float scale,
+                        cudaStream_t stream);
 
 /*
  * Largest scratch, in bytes, that fa_bwd_noalloc can use (32 MiB). A problem
@@ -218,9 +264,11 @@ const char* fa_status_string(fa_status s);
 
 /*
  * Device status word of the current device, then cleared. 0 when no kernel
- * has given up on a bounded wait since the last call. Otherwise the low byte
- * is an fa_status (FA_ERR_TIMEOUT) and bits 8.. name the wait that gave up.
- * Synchronises the device. Returns -1 if the word could not be read.
+ * has given up on a bounded wait or met bad packed-batch offsets since the
+ * last call. Otherwise the low byte is an fa_status (FA_ERR_TIMEOUT, or
+ * FA_ERR_INVALID_ARG for offsets) and bits 8.. name the wait that gave up
+ * (64: the offsets check). Synchronises the device. Returns -1 if the word
+ * could not be read.
  */
 int fa_last_device_status(void);
 

@@ -25,7 +25,7 @@ int main(void) {
   CHECK(fa_decode_workspace_size(16, 32, 8, 1, 16384, 128, 0) > 0);
   CHECK(fa_decode_workspace_size(1, 8, 1, 4, 100, 128, 0) == 0);  /* 32 query rows per KV head */
   CHECK(fa_fwd(NULL, P, P, P, (float*)P, 1, 2, 2, 128, 64, 0, 0.125f, 0) == FA_ERR_INVALID_ARG);
-  CHECK(fa_fwd(P, P, P, P, (float*)P, 1, 2, 2, 128, 96, 0, 0.125f, 0) == FA_ERR_UNSUPPORTED);
+  CHECK(fa_fwd(P, P, P, P, (float*)P, 1, 2, 2, 128, 80, 0, 0.125f, 0) == FA_ERR_UNSUPPORTED);
   CHECK(fa_fwd((char*)P + 2, P, P, P, (float*)P, 1, 2, 2, 128, 64, 0, 0.125f, 0) == FA_ERR_MISALIGNED);
   {
     size_t ws = fa_bwd_workspace_size(1, 2, 2, 128, 64);

@@ -68,8 +68,10 @@ def test_fwd_rejects_bad_arguments(lib):
     assert fwd(lib, scale=-1.0) == 1
     assert fwd(lib, scale=float("inf")) == 1
     assert fwd(lib, scale=float("nan")) == 1
-    assert fwd(lib, d=96) == 2
-    assert fwd(lib, d=256) == 2
+    assert fwd(lib, d=80) == 2
+    assert fwd(lib, d=112) == 2
+    assert fwd(lib, d=320) == 2
+    assert fwd(lib, d=160) == 2
     assert fwd(lib, B=65536, Hq=256, Hkv=256, N=16384) == 2  # grid of more than 2^31 - 1 CTAs
     assert fwd(lib, q=P + 8) == 3
     assert fwd(lib, lse=P + 4) == 3
@@ -81,6 +83,8 @@ def test_bwd_rejects_bad_arguments(lib):
         return lib.fa_bwd(P, P, P, P, P, P, dq, P, P, ws_ptr, ws_bytes, 1, 2, 2, 128, d, 0, 0.125, None)
     assert bwd(dq=None) == 1
     assert bwd(d=80) == 2
+    assert bwd(d=192) == 2   # the wide-head kernels are forward only
+    assert bwd(d=256) == 2
     assert bwd(ws_ptr=None) == 4
     assert bwd(ws_bytes=ws - 1) == 4
     assert bwd(dq=P + 2) == 3
@@ -99,13 +103,40 @@ def test_bwd_noalloc_reports_argument_errors_before_its_size_limit(lib):
     assert nb(scale=0.0) == 1                  # bad scale
     assert nb(scale=float("nan")) == 1
     assert nb(sizes=(2, 33, 8, 8192, 128)) == 1  # Hq % Hkv != 0
-    assert nb(sizes=(2, 32, 8, 8192, 96)) == 2   # head dimension
+    assert nb(sizes=(2, 32, 8, 8192, 80)) == 2   # head dimension
     assert nb(dq=P + 2) == 3                   # misaligned
     assert nb() == 4                           # only then: larger than the built-in scratch
     # the limit is exact: 2 x 64 heads x 992 rows x 64 needs exactly 32 MiB
     # (launching would need a GPU, so only the size query is checked here)
     assert lib.fa_bwd_workspace_size(2, 64, 16, 992, 64) == 32 * 1024 * 1024
     assert lib.fa_bwd_workspace_size(1, 129, 129, 992, 64) > 32 * 1024 * 1024
+
+
+def test_varlen_rejects_bad_arguments(lib):
+    """Host-side checks of the packed entry points (the offsets themselves
+    live on the device and are checked by the kernels)."""
+    def fv(cu=P, B=2, Hq=2, Hkv=2, T=300, maxlen=200, d=64, lse=P, scale=0.125):
+        return lib.fa_fwd_varlen(P, P, P, P, lse, cu, B, Hq, Hkv, T, maxlen, d, 1, scale, None)
+    assert fv(cu=None) == 1
+    assert fv(lse=None) == 1
+    assert fv(T=-1) == 1
+    assert fv(Hq=3) == 1
+    assert fv(d=80) == 2
+    assert fv(scale=0.0) == 1
+    assert fv(cu=P + 2) == 3                  # offsets must be 4-byte aligned
+    assert fv(T=0) == 0 and fv(maxlen=0) == 0  # every sequence empty: nothing to do
+    ws = lib.fa_bwd_varlen_workspace_size(2, 2, 2, 300, 200, 64)
+    assert ws > 0
+    def bv(wsp=P, ws_bytes=ws, cu=P, d=64):
+        return lib.fa_bwd_varlen(P, P, P, P, P, P, P, P, P, cu, wsp, ws_bytes, 2, 2, 2, 300, 200, d, 1, 0.125, None)
+    assert bv(cu=None) == 1
+    assert bv(wsp=None) == 4
+    assert bv(ws_bytes=ws - 1) == 4
+    assert bv(d=80) == 2
+    # linear in the tokens and in the longest sequence
+    a = lib.fa_bwd_varlen_workspace_size(2, 2, 2, 4096, 2048, 128)
+    b = lib.fa_bwd_varlen_workspace_size(2, 2, 2, 8192, 4096, 128)
+    assert b <= 2 * a + 512
 
 
 def test_fp8_rejects_bad_arguments(lib):

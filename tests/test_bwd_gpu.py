@@ -47,7 +47,7 @@ def test_tiny_workload(causal):
 
 
 @pytest.mark.parametrize("N", [1, 17, 127, 128, 129, 255, 257, 383, 1000])
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("causal", [False, True])
 def test_edge_sizes(N, d, causal):
     dev, host = make_inputs(1, 2, 2, N, d, seed=2000 + N + d)

@@ -4,54 +4,33 @@
   float32 block scales must equal the oracle quantiser's bit for bit (the
   rotated values are exact fp64 sums rounded once to fp32 on both sides).
 * The FP8 forward is compared with the oracle's fp64 emulation of the same
-  steps. The kernel's scores come from the FP8 tensor-core product, which is
-  not exact to fp64 (relative error of order 1e-4 in the log2-domain scores);
-  near an e4m3 rounding boundary that flips P's code by one step (up to 1/8
-  of its value), and in a peaked row one flip moves O visibly. The emulation
-  itself moves by the same amount (0.06 max, 3e-4 RMS on a 385-row case) when
-  its scores are perturbed by 1e-4 relative. So the bound per element is
-  2e-2 + 1/4 * Pmax_i * max|V| (one step on the row's two largest
-  probabilities; Pmax_i the exact largest probability of row i) and LSE must
-  agree within 1e-2. The RMS of kernel - emulation must stay under half the
-  emulation's own RMS error against exact attention, and the kernel's RMS
-  error against exact attention may exceed the emulation's by at most 10 %:
-  the kernel must be as accurate as the emulated method, not equal to it.
-* The kernel's error against exact fp64 attention is reported next to the
-  naive per-tensor FP8 baseline's, and must not be worse.
+  steps ("FlashAttention-3: Fast and Accurate Attention with Asynchrony and
+  Low-precision", abstract: block quantisation and incoherent processing).
+  What may differ, and the gates derived from it:
+  - O is bf16 (half an ulp: at most 2^-9 |O|), the emulation fp64: on the
+    test inputs this is an RMS of about 3 % of the emulation's own RMS error
+    against exact attention.
+  - The kernel forms P~ w in fp32 (one FFMA, MUFU ex2.approx, one FMUL);
+    its scores agree with the emulation's to about 1e-6 (LSE within 1e-5 on
+    every case measured). Where P~ w of one key lies that close to an e4m3
+    rounding boundary the two sides pick neighbouring codes: O_ic moves by
+    at most 2^-3 P_ij |V_jc| per flipped key (e4m3 has 3 mantissa bits).
+  Gates: per element |O - O_emu| <= 2e-2 + 1/4 M_ic, with M_ic the largest
+  single term max_j P_ij |V_jc| of the row's own sum (two flips on its
+  largest terms; the floor covers the bf16 half-ulp and flips of small
+  terms); LSE within 1e-4 (ten times the largest measured gap); and the RMS
+  of O - O_emu at most 0.1 of the emulation's RMS error against exact
+  attention over all rows but the max(2, 0.1 %) rows with the largest
+  difference: a flip of a row's dominant probability moves a whole row (one
+  such event in a 400-row case alone is 0.34 of the RMS), and those rows are
+  still held to the element bound.
+* The kernel must be as accurate as the method: its RMS error against exact
+  fp64 attention may exceed the 128-key emulation's, and the single-tile
+  emulation's (P rounded against the row's final maximum), by at most 10 %.
+* Its error against exact fp64 attention is reported next to the naive
+  per-tensor FP8 baseline's (rounding the unnormalised P~ = exp(S - m), and
+  the normalised probabilities), and must not be worse than either.
 """
-
-FP8_LSE_MAX_ABS = 1e-2
-
-
-def row_pmax(q, k, scale, causal, lse, chunk=2048):
-    """Largest softmax probability of each row: exp(max_j S_ij - LSE_i)."""
-    B, H, N, d = q.shape
-    g = H // k.shape[1]
-    out = np.empty((B, H, N))
-    for b in range(B):
-        for h in range(H):
-            for r0 in range(0, N, chunk):
-                r1 = min(N, r0 + chunk)
-                s = scale * (q[b, h, r0:r1] @ k[b, h // g].T)
-                if causal:
-                    s = np.where(np.arange(N)[None, :] > np.arange(r0, r1)[:, None], -np.inf, s)
-                out[b, h, r0:r1] = np.exp(s.max(axis=1) - lse[b, h, r0:r1])
-    return out
-
-
-def check_against_emulation(o, lse, o_emu, lse_emu, q, k, v, causal, scale):
-    exact, lse_exact = oracle.attention_forward(q, k, v, causal, scale)
-    pmax = row_pmax(q, k, scale, causal, lse_exact)
-    bound = O_MAX_ABS + 0.25 * pmax[..., None] * np.abs(v).max()
-    err = np.abs(o - o_emu)
-    assert np.all(err <= bound), f"{np.count_nonzero(err > bound)} elements past the flip bound, max {err.max()}"
-    rms_diff = math.sqrt(np.mean((o - o_emu) ** 2))
-    rms_emu = math.sqrt(np.mean((o_emu - exact) ** 2))
-    rms_gpu = math.sqrt(np.mean((o - exact) ** 2))
-    assert rms_diff <= 0.5 * rms_emu, (rms_diff, rms_emu)
-    assert rms_gpu <= 1.1 * rms_emu + 1e-4, (rms_gpu, rms_emu)
-    assert np.max(np.abs(lse - lse_emu)) <= FP8_LSE_MAX_ABS, np.max(np.abs(lse - lse_emu))
-    return exact
 
 import math
 
@@ -65,6 +44,64 @@ from synthetic import WORKLOADS, sign_vector
 from _helpers import O_MAX_ABS, make_inputs, to_f64
 
 pytestmark = pytest.mark.gpu
+
+
+FP8_LSE_MAX_ABS = 1e-4
+FP8_RMS_RATIO = 0.1
+FLIP_ROW_SHARE = 1e-3
+
+
+def attended_max(q, k, v, scale, causal, lse, top=32, chunk=1024):
+    """Upper bound of M_ic = max_j P_ij |V_jc| (the largest single term of
+    O_ic's sum): exact over each row's `top` most probable keys, and
+    P_(top+1) max_j |V_jc| for all the others."""
+    B, H, N, d = q.shape
+    g = H // k.shape[1]
+    out = np.empty((B, H, N, d))
+    for b in range(B):
+        for h in range(H):
+            vabs = np.abs(v[b, h // g])
+            vmax = vabs.max(axis=0)
+            kk = min(top, N)
+            for r0 in range(0, N, chunk):
+                r1 = min(N, r0 + chunk)
+                s = scale * (q[b, h, r0:r1] @ k[b, h // g].T)
+                if causal:
+                    s = np.where(np.arange(N)[None, :] > np.arange(r0, r1)[:, None], -np.inf, s)
+                p = np.exp(s - lse[b, h, r0:r1, None])
+                if kk < N:
+                    idx = np.argpartition(-p, kk - 1, axis=1)[:, :kk]
+                else:
+                    idx = np.tile(np.arange(N), (r1 - r0, 1))
+                ptop = np.take_along_axis(p, idx, axis=1)
+                m = np.max(ptop[:, :, None] * vabs[idx], axis=1)
+                if kk < N:
+                    rest = -np.partition(-p, kk, axis=1)[:, kk]
+                    m = np.maximum(m, rest[:, None] * vmax[None, :])
+                out[b, h, r0:r1] = m
+    return out
+
+
+def check_against_emulation(o, lse, o_emu, lse_emu, q, k, v, causal, scale, sigma=None):
+    exact, lse_exact = oracle.attention_forward(q, k, v, causal, scale)
+    M = attended_max(q, k, v, scale, causal, lse_exact)
+    bound = O_MAX_ABS + 0.25 * M
+    err = np.abs(o - o_emu)
+    assert np.all(err <= bound), f"{np.count_nonzero(err > bound)} elements past the flip bound, max {err.max()}"
+    assert np.max(np.abs(lse - lse_emu)) <= FP8_LSE_MAX_ABS, np.max(np.abs(lse - lse_emu))
+    d = o.shape[-1]
+    row_ms = np.mean((o - o_emu).reshape(-1, d) ** 2, axis=1)
+    drop = max(2, int(math.ceil(FLIP_ROW_SHARE * row_ms.size)))
+    kept = np.sort(row_ms)[:max(1, row_ms.size - drop)]
+    rms_diff = math.sqrt(np.mean(kept))
+    rms_emu = math.sqrt(np.mean((o_emu - exact) ** 2))
+    rms_gpu = math.sqrt(np.mean((o - exact) ** 2))
+    assert rms_diff <= FP8_RMS_RATIO * rms_emu, (rms_diff, rms_emu)
+    assert rms_gpu <= 1.1 * rms_emu + 1e-4, (rms_gpu, rms_emu)
+    o_one, _ = oracle.fp8_attention_forward(q, k, v, causal, scale, sigma, tile=1 << 30)
+    rms_one = math.sqrt(np.mean((o_one - exact) ** 2))
+    assert rms_gpu <= 1.1 * rms_one + 1e-4, (rms_gpu, rms_one)
+    return exact
 
 
 def up1024(x):
@@ -129,7 +166,8 @@ def test_forward_matches_emulation(causal, N, Hq, Hkv):
     o_emu, lse_emu = oracle.fp8_attention_forward(host["q"], host["k"], host["v"], causal, d ** -0.5,
                                                   sign_vector(seed, d))
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
-    check_against_emulation(o, lse, o_emu, lse_emu, host["q"], host["k"], host["v"], causal, d ** -0.5)
+    check_against_emulation(o, lse, o_emu, lse_emu, host["q"], host["k"], host["v"], causal, d ** -0.5,
+                            sign_vector(seed, d))
 
 
 def test_forward_without_rotation_matches_emulation():
@@ -137,7 +175,7 @@ def test_forward_without_rotation_matches_emulation():
     dev, host = make_inputs(1, 2, 2, 640, d, seed=71, outlier_rate=0.001, with_dout=False)
     o, lse, _ = run_fp8(dev, False, 5, False)
     o_emu, lse_emu = oracle.fp8_attention_forward(host["q"], host["k"], host["v"], False, d ** -0.5, None)
-    check_against_emulation(o, lse, o_emu, lse_emu, host["q"], host["k"], host["v"], False, d ** -0.5)
+    check_against_emulation(o, lse, o_emu, lse_emu, host["q"], host["k"], host["v"], False, d ** -0.5, None)
 
 
 def test_full_fp8_workload_sampled_error_report():
@@ -153,17 +191,20 @@ def test_full_fp8_workload_sampled_error_report():
     sigma = sign_vector(seed, w.d)
     heads = [(0, 0), (0, w.Hq - 1)]
     naive_all = oracle.naive_fp8_attention_forward(host["q"], host["k"], host["v"], False, w.scale, heads=heads)
+    naive_norm = oracle.naive_fp8_attention_forward(host["q"], host["k"], host["v"], False, w.scale, heads=heads,
+                                                    p_form="normalised")
     for _, h in heads:
         sl = slice(h, h + 1)
         q, k, v = host["q"][:, sl], host["k"][:, sl], host["v"][:, sl]
         o_emu, lse_emu = oracle.fp8_attention_forward(q, k, v, False, w.scale, sigma)
-        exact = check_against_emulation(o[:, sl], lse[:, sl], o_emu, lse_emu, q, k, v, False, w.scale)
-        naive = naive_all[:, sl]  # per-tensor scales: amax over every head
+        exact = check_against_emulation(o[:, sl], lse[:, sl], o_emu, lse_emu, q, k, v, False, w.scale, sigma)
         rmse_ours = math.sqrt(np.mean((o[:, sl] - exact) ** 2))
-        rmse_naive = math.sqrt(np.mean((naive - exact) ** 2))
-        print(f"head {h}: RMSE fp8 kernel {rmse_ours:.3e}, naive per-tensor fp8 {rmse_naive:.3e}, "
-              f"ratio {rmse_naive / rmse_ours:.2f}")
-        assert rmse_ours < rmse_naive
+        rmse_naive = math.sqrt(np.mean((naive_all[:, sl] - exact) ** 2))   # per-tensor scales: amax over every head
+        rmse_norm = math.sqrt(np.mean((naive_norm[:, sl] - exact) ** 2))
+        print(f"head {h}: RMSE fp8 kernel {rmse_ours:.3e}; naive per-tensor fp8 {rmse_naive:.3e} "
+              f"(ratio {rmse_naive / rmse_ours:.2f}), with normalised P {rmse_norm:.3e} "
+              f"(ratio {rmse_norm / rmse_ours:.2f})")
+        assert rmse_ours < rmse_naive and rmse_ours < rmse_norm
 
 
 @pytest.mark.parametrize("rotate", [True, False])

@@ -40,7 +40,7 @@ def test_tiny_workload(causal):
 
 
 @pytest.mark.parametrize("N", [1, 17, 127, 128, 129, 255, 256, 257, 383, 1000])
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128, 192, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_edge_sizes(N, d, causal):
     dev, host = make_inputs(1, 2, 2, N, d, seed=1000 + N + d, with_dout=False)
@@ -56,6 +56,19 @@ def test_gqa_small(Hq, Hkv, causal):
     o, lse = run_fwd(dev, causal)
     o_ref, lse_ref = oracle.attention_forward(host["q"], host["k"], host["v"], causal, 128 ** -0.5)
     check(o, lse, o_ref, lse_ref)
+
+
+@pytest.mark.parametrize("d", [192, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_wide_heads_gqa_and_many_key_tiles(d, causal):
+    """The wide-head kernel (one query tile, 64-key tiles, two score
+    buffers) over many key tiles with GQA and a ragged end, plus large
+    scores that make the running maximum move."""
+    dev, host = make_inputs(2, 4, 2, 1100, d, seed=91 + d, with_dout=False)
+    for scale in (d ** -0.5, 0.5):
+        o, lse = run_fwd(dev, causal, scale)
+        o_ref, lse_ref = oracle.attention_forward(host["q"], host["k"], host["v"], causal, scale)
+        check(o, lse, o_ref, lse_ref)
 
 
 def test_scale_and_large_scores():
