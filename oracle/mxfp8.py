@@ -34,9 +34,10 @@ Attention (readings, stated here because the sources give none):
   FP8 path (the 1/d folds into the softmax scale).
 * O = P V contracts over the keys: V is quantised in blocks of 32 keys of each
   column, and so is P, per row, tile by tile.
-* Keys are visited 128 at a time with an exact running max m (so P <= 1):
-  P = exp2(c S - m) rounded to float32, then MX-quantised along the keys of
-  the tile; the row sum l accumulates the unquantised P; O = acc / l.
+* Keys are visited 128 at a time with a running max m (exact by default, so
+  P <= 1; optionally raised only past tau, as the bf16 path defers its
+  rescale): P = exp2(c S - m) rounded to float32, then MX-quantised along the
+  keys of the tile; the row sum l accumulates the unquantised P; O = acc / l.
 
 Parity pins (``tests/test_oracle_mxfp8_pins.py``): closed-form blocks from the
 conversion rule (scale, clamp, zero block, where the two rules differ), the
@@ -111,10 +112,13 @@ def mx_roundtrip(x, axis: int = -1, block: int = MX_BLOCK, rule: str = "ocp") ->
 
 
 def mxfp8_attention_forward(q, k, v, causal: bool, scale: float, sigma=None, tile: int = 128,
-                            quantize_p: bool = True, rule: str = "ocp"):
+                            quantize_p: bool = True, rule: str = "ocp", tau: float = 0.0):
     """Emulate the MXFP8 forward (readings in the module docstring) in
     float64, with the scale rule of ``mx_quantize``. ``quantize_p=False``
     leaves P unquantised (used to pin the score and softmax assembly).
+    ``tau`` > 0 lets a row keep its running max until a tile's max exceeds
+    it by more than tau (log2 units), as the bf16 path's deferred rescale
+    does; P then reaches up to 2^tau, which MX block scales absorb.
     Returns (O, LSE) with LSE in natural log."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
@@ -146,7 +150,8 @@ def mxfp8_attention_forward(q, k, v, causal: bool, scale: float, sigma=None, til
                 s = c * (qh[b, h] @ kh[b, kvh, j0:j1].T)
                 if causal:
                     s = np.where(np.arange(j0, j1)[None, :] > rows[:, None], -np.inf, s)
-                m_new = np.maximum(m, np.max(s, axis=1))
+                tmax = np.max(s, axis=1)
+                m_new = np.where(tmax > m + tau, np.maximum(m, tmax), m)
                 m_use = np.where(np.isneginf(m_new), 0.0, m_new)
                 alpha = np.where(np.isneginf(m), 0.0, np.exp2(m - m_use))
                 p = np.exp2(s - m_use[:, None]).astype(np.float32).astype(np.float64)

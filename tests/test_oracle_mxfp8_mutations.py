@@ -17,6 +17,8 @@ import test_oracle_mxfp8_pins as pins  # noqa: E402
 SRC = open(mxmod.__file__).read().replace("from .fp8 import", "from oracle.fp8 import")
 
 MUTATIONS = [
+    ("max raised on every increase despite tau", "m_new = np.where(tmax > m + tau, np.maximum(m, tmax), m)",
+     "m_new = np.maximum(m, tmax)", [pins.test_mxfp8_deferred_max_two_tile_closed_form]),
     ("shared exponent off by one", "e = E - 1 - E4M3_EMAX", "e = E - E4M3_EMAX",
      [pins.test_closed_form_blocks]),
     ("fit rule at the boundary", "e = e + (m > 0.875)", "e = e + (m >= 0.875)",

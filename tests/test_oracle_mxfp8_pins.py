@@ -200,3 +200,44 @@ def test_accuracy_on_the_fp8_input_recipe(seed):
     assert e_fit < e_ocp
     assert e_fit < 1.1 * e_64
     assert e_fit < 0.1 * rms(exact)
+
+
+def test_mxfp8_deferred_max_two_tile_closed_form():
+    """Two keys visited one per tile, log2-domain scores 0 and 0.5 (scale =
+    ln 2; Q = e_0, K_1 = 0.5 e_0: codes 256 and 256 with exact block scales).
+    With tau = 8 the second tile's max does not raise m = 0, so that tile's P
+    is 2^0.5, one block whose exponent is floor(log2 2^0.5) - 8 = -8 (both
+    rules: the significand 1.414 is below 1.75): code 362.04 -> 352 (quantum
+    32), P^ = 1.375, O = (V_0 + 1.375 V_1) / (1 + 2^0.5). With tau = 0 every
+    code is exact and O is the softmax's. V's columns are exact in MX (blocks
+    of 32 keys: amax 2, 2, 2, 0.25)."""
+    q = np.zeros((1, 1, 2, 32))
+    q[..., 0] = 1.0
+    k = np.zeros((1, 1, 2, 32))
+    k[0, 0, 1, 0] = 0.5
+    v = np.zeros((1, 1, 2, 32))
+    v[0, 0, 0, :4] = [2.0, -1.0, 0.5, 0.0]
+    v[0, 0, 1, :4] = [1.0, 2.0, -2.0, 0.25]
+    for rule in ("ocp", "fit"):
+        o8, _ = oracle.mxfp8_attention_forward(q, k, v, False, math.log(2.0), None, tile=1, rule=rule, tau=8.0)
+        want = (v[0, 0, 0] + 1.375 * v[0, 0, 1]) / (1 + 2 ** 0.5)
+        np.testing.assert_allclose(o8[0, 0, 0], want, rtol=1e-7, atol=1e-12)   # P and l in float32
+        o0, _ = oracle.mxfp8_attention_forward(q, k, v, False, math.log(2.0), None, tile=1, rule=rule, tau=0.0)
+        exact = (2 ** -0.5 * v[0, 0, 0] + v[0, 0, 1]) / (1 + 2 ** -0.5)
+        np.testing.assert_allclose(o0[0, 0, 0], exact, rtol=1e-7, atol=1e-12)
+
+
+def test_mxfp8_deferred_max_keeps_accuracy_and_lse():
+    """tau = 8 rounds different multiples of the same P; the LSE does not
+    depend on when m is raised (up to P's float32 rounding), and the accuracy
+    against exact attention stays within 10 %."""
+    rng = np.random.default_rng(41)
+    q, k, v = (rng.standard_normal((1, 2, 384, 64)) for _ in range(3))
+    exact, _ = oracle.attention_forward(q, k, v, True, 0.125)
+    o0, l0 = oracle.mxfp8_attention_forward(q, k, v, True, 0.125, rule="fit", tau=0.0)
+    o8, l8 = oracle.mxfp8_attention_forward(q, k, v, True, 0.125, rule="fit", tau=8.0)
+    rms = lambda a: math.sqrt(np.mean(a ** 2))
+    # the same except for P's float32 rounding at a different scale
+    np.testing.assert_allclose(l0, l8, rtol=0, atol=1e-6)
+    assert abs(rms(o0 - exact) - rms(o8 - exact)) <= 0.1 * rms(o0 - exact)
+    assert rms(o0 - o8) < 0.5 * rms(o0 - exact)
