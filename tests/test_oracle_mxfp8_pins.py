@@ -219,10 +219,10 @@ def test_mxfp8_deferred_max_two_tile_closed_form():
     v[0, 0, 0, :4] = [2.0, -1.0, 0.5, 0.0]
     v[0, 0, 1, :4] = [1.0, 2.0, -2.0, 0.25]
     for rule in ("ocp", "fit"):
-        o8, _ = oracle.mxfp8_attention_forward(q, k, v, False, math.log(2.0), None, tile=1, rule=rule, tau=8.0)
+        o8, _ = mx.mxfp8_attention_forward(q, k, v, False, math.log(2.0), None, tile=1, rule=rule, tau=8.0)
         want = (v[0, 0, 0] + 1.375 * v[0, 0, 1]) / (1 + 2 ** 0.5)
         np.testing.assert_allclose(o8[0, 0, 0], want, rtol=1e-7, atol=1e-12)   # P and l in float32
-        o0, _ = oracle.mxfp8_attention_forward(q, k, v, False, math.log(2.0), None, tile=1, rule=rule, tau=0.0)
+        o0, _ = mx.mxfp8_attention_forward(q, k, v, False, math.log(2.0), None, tile=1, rule=rule, tau=0.0)
         exact = (2 ** -0.5 * v[0, 0, 0] + v[0, 0, 1]) / (1 + 2 ** -0.5)
         np.testing.assert_allclose(o0[0, 0, 0], exact, rtol=1e-7, atol=1e-12)
 
@@ -234,8 +234,8 @@ def test_mxfp8_deferred_max_keeps_accuracy_and_lse():
     rng = np.random.default_rng(41)
     q, k, v = (rng.standard_normal((1, 2, 384, 64)) for _ in range(3))
     exact, _ = oracle.attention_forward(q, k, v, True, 0.125)
-    o0, l0 = oracle.mxfp8_attention_forward(q, k, v, True, 0.125, rule="fit", tau=0.0)
-    o8, l8 = oracle.mxfp8_attention_forward(q, k, v, True, 0.125, rule="fit", tau=8.0)
+    o0, l0 = mx.mxfp8_attention_forward(q, k, v, True, 0.125, rule="fit", tau=0.0)
+    o8, l8 = mx.mxfp8_attention_forward(q, k, v, True, 0.125, rule="fit", tau=8.0)
     rms = lambda a: math.sqrt(np.mean(a ** 2))
     # the same except for P's float32 rounding at a different scale
     np.testing.assert_allclose(l0, l8, rtol=0, atol=1e-6)
