@@ -291,13 +291,15 @@ __device__ __forceinline__ float ex2(float x) {
 // 2^x evaluated on the FMA pipe instead of the MUFU unit, so that a share of
 // the softmax exponentials can run beside the MUFU ones. Range reduction:
 // x = j + f with j = round-to-nearest(x) (read from the low mantissa bits of
-// x + 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose
-// coefficients were fitted for minimal maximum relative error
-// (fit_exp2_poly.py: 7.5e-5, below bf16's 2^-9 rounding of P); 2^j is added
-// to the exponent bits. Valid for x <= 64; inputs below -126 (including -inf
-// from masked scores) are clamped, giving at most 2^-125.
+// x + 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a cubic whose constant term
+// is exactly 1 (so 2^0 = 1: a row's largest score must give P = 1 exactly)
+// and whose other coefficients were fitted for minimal maximum relative
+// error (fit_exp2_poly.py: 1.01e-4, far below e4m3's 2^-4 and bf16's 2^-9
+// rounding of P); 2^j is added to the exponent bits. Valid for x <= 64;
+// inputs below -126 (including -inf from masked scores) are clamped, giving
+// at most 2^-125.
 __device__ __forceinline__ float exp2_poly(float x) {
-  constexpr float C0 = 0x1.fff692p-1f, C1 = 0x1.62f31ap-1f, C2 = 0x1.f0de1cp-3f, C3 = 0x1.c3f76p-5f;
+  constexpr float C0 = 0x1p+0f, C1 = 0x1.62f5fap-1f, C2 = 0x1.f00c4ep-3f, C3 = 0x1.c2a216p-5f;
   constexpr float SHIFT = 12582912.0f;  // 1.5 * 2^23
   x = fmaxf(x, -126.0f);
   const float t = __fadd_rn(x, SHIFT);

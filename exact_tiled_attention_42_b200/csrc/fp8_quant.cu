@@ -19,21 +19,10 @@
 // time, d/32 consecutive elements per lane. HBM-bound.
 #include "common.cuh"
 #include "kernels.h"
+#include "rotation.cuh"
 
 namespace fa {
 namespace {
-
-constexpr uint64_t SM_GAMMA = 0x9E3779B97F4A7C15ull;
-
-__device__ __forceinline__ uint64_t splitmix_mix(uint64_t z) {
-  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-  return z ^ (z >> 31);
-}
-// Output number `i` (0-based) of SplitMix64 seeded with `seed`.
-__device__ __forceinline__ uint64_t splitmix_at(uint64_t seed, uint64_t i) {
-  return splitmix_mix(seed + (i + 1) * SM_GAMMA);
-}
 
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
   uint16_t r;
@@ -53,11 +42,7 @@ __global__ void __launch_bounds__(256) fp8_quant_kernel(const Fp8Params p) {
   __shared__ float warp_max[8];
 
   float sig[E];
-  if (rot) {
-    const uint64_t key = splitmix_at(p.rotation_seed, 5);
-#pragma unroll
-    for (int e = 0; e < E; ++e) sig[e] = (splitmix_at(key, lane * E + e) >> 63) ? -1.f : 1.f;
-  }
+  if (rot) rotation_signs<E>(sig, p.rotation_seed, lane);
 
   float y[8][E];
   float amax = 0.f;
@@ -71,30 +56,7 @@ __global__ void __launch_bounds__(256) fp8_quant_kernel(const Fp8Params p) {
       double x[E];
 #pragma unroll
       for (int e = 0; e < E; ++e) x[e] = static_cast<double>(__uint_as_float(static_cast<uint32_t>(row[e]) << 16));
-      if (rot) {
-#pragma unroll
-        for (int e = 0; e < E; ++e) x[e] *= sig[e];
-        // in-lane butterflies (h < E), then across lanes (h >= E)
-#pragma unroll
-        for (int h = 1; h < E; h <<= 1)
-#pragma unroll
-          for (int e = 0; e < E; ++e)
-            if (!(e & h)) {
-              const double a = x[e], b = x[e + h];
-              x[e] = a + b;
-              x[e + h] = a - b;
-            }
-#pragma unroll
-        for (int h = E; h < D; h <<= 1) {
-          const int lm = h / E;
-          const bool upper = (lane & lm) != 0;
-#pragma unroll
-          for (int e = 0; e < E; ++e) {
-            const double other = __shfl_xor_sync(0xffffffffu, x[e], lm);
-            x[e] = upper ? other - x[e] : x[e] + other;
-          }
-        }
-      }
+      if (rot) hadamard_row<E, D>(x, sig, lane);
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         y[rr][e] = __double2float_rn(x[e]);

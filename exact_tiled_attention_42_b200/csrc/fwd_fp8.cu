@@ -44,8 +44,11 @@ constexpr float P_LIFT = 256.f;
 constexpr float TAU = 0.8f;
 static_assert(P_LIFT * 1.7411011f <= 448.f, "2^TAU * P_LIFT must stay within e4m3's range");
 // Of every 8 groups of 4 scores, this many take their exponentials on the FMA
-// pipe (exp2_poly) instead of MUFU.
-constexpr int POLY_GROUPS = 0;
+// pipe (exp2_poly) instead of MUFU: the two query tiles' 2 x 128 x 128
+// exponentials per key tile need 2048 MUFU cycles against about 1080 of e4m3
+// MMA. Measured on the FP8 workload (forward alone): 0 -> 1205, 2 -> 1279,
+// 3 -> 1186 TFLOP/s.
+constexpr int POLY_GROUPS = 2;
 
 // exp2_poly on two values with packed FMA-pipe arithmetic.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
@@ -288,7 +291,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int off = 16; off > 0; off >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
     const float wlift = P_LIFT / vmax;
     const float crow = p.score_log2 * sQs[min(qrow, p.N - 1) >> 6];
-    float m = -INFINITY;
+    float m = -INFINITY;  // running max of the log2-domain scores, as m + mlo (mlo: m's rounding residual)
+    float mlo = 0.f;
     float l = 0.f;
     bool ok = n > 0;
     for (int j = 0; ok && j < n; ++j) {
@@ -324,20 +328,27 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (kv0 + c >= lim) s[c] = -INFINITY;
       }
       // row maxima of the two key halves (three-input max)
-      const float mlo = row_max<64>(s);
-      const float mhi = row_max<64>(s + 64);
-      const float tile_max = fmaxf(mlo * f0, mhi * f1);
+      const float smax0 = row_max<64>(s);
+      const float smax1 = row_max<64>(s + 64);
+      const float t0 = smax0 * f0, t1 = smax1 * f1;
+      const bool top1 = t1 > t0;
+      const float tile_max = top1 ? t1 : t0;
+      // exact residual of the largest product: f smax = tile_max + tile_lo
+      const float tile_lo = tile_max > -INFINITY ? (top1 ? fmaf(smax1, f1, -t1) : fmaf(smax0, f0, -t0)) : 0.f;
       if (j == 0) {
         m = tile_max;
+        mlo = tile_lo;
       } else {
         // a row raises its max only past TAU; the warp rescales O in tensor
         // memory when any of its rows did (alpha = 1 for the others)
         const bool raise = tile_max > m + TAU;
         if (__any_sync(0xffffffffu, raise)) {
-          const float m_new = raise ? fmaxf(m, tile_max) : m;
-          const float alpha = ex2(m - m_new);
+          const float m_new = raise ? tile_max : m;
+          const float mlo_new = raise ? tile_lo : mlo;
+          const float alpha = ex2((m - m_new) + (mlo - mlo_new));
           l *= alpha;
           m = m_new;
+          mlo = mlo_new;
 #pragma unroll
           for (int c = 0; c < D; c += 16) {
             uint32_t r[16];
@@ -354,16 +365,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       // multiply, but P~ = 1 for a row's largest key, and 2^(log2 w) is not
       // exactly w: where w sits on an e4m3 rounding tie -- block scales are
       // ratios of short bf16 values, so it can -- the code would flip.)
+      // x = fl(fma(s, f, -m) - mlo): the fused product-minus-max is exact at
+      // the key that set the max (it equals mlo there), so that key gets
+      // x = 0 and P = 1 exactly whatever the compiler fuses (otherwise the
+      // product's rounding residual survives and P w can round off an e4m3
+      // tie the other way)
       const float nm = (m == -INFINITY) ? 0.f : -m;
       const float2 f0v = make_float2(f0, f0), f1v = make_float2(f1, f1), nmv = make_float2(nm, nm);
+      const float2 nlov = make_float2(-mlo, -mlo);
       const float2 w0v = make_float2(w0, w0), w1v = make_float2(w1, w1);
       float2 lsum[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const bool hi = i >= 16;
-        const float2 x01 = __ffma2_rn(make_float2(s[4 * i], s[4 * i + 1]), hi ? f1v : f0v, nmv);
-        const float2 x23 = __ffma2_rn(make_float2(s[4 * i + 2], s[4 * i + 3]), hi ? f1v : f0v, nmv);
+        const float2 x01 = __fadd2_rn(__ffma2_rn(make_float2(s[4 * i], s[4 * i + 1]), hi ? f1v : f0v, nmv), nlov);
+        const float2 x23 = __fadd2_rn(__ffma2_rn(make_float2(s[4 * i + 2], s[4 * i + 3]), hi ? f1v : f0v, nmv), nlov);
         float2 a01, a23;
         if ((i & 7) < POLY_GROUPS) {
           a01 = exp2_poly2(x01);
@@ -415,7 +432,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         bulk_commit();
         bulk_wait_read0();
       }
-      if (qrow < p.N) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(l)) * LN2;
+      if (qrow < p.N) p.lse[static_cast<size_t>(bh) * p.N + qrow] = ((m + mlo) + __log2f(l)) * LN2;
     }
   }
 

@@ -1,4 +1,4 @@
-"""The FMA-pipe exp2 used for part of the softmax exponentials: its
+"""The FMA-pipe exp2 used for part of the FP8 softmax's exponentials: its
 coefficients reproduce from the committed fit, and a step-by-step float32
 emulation of the device function (same range reduction and Horner steps; an
 fp32 FMA is emulated as the exact product-sum rounded once) stays within the
@@ -40,7 +40,8 @@ def emulate(x):
 def test_coefficients_match_the_fit():
     fitted = fit_exp2_poly.fit()
     np.testing.assert_array_equal(np.array(device_coefficients(), np.float32), fitted)
-    assert fit_exp2_poly.max_rel_error(fitted) < 1e-4
+    assert fitted[0] == 1.0
+    assert fit_exp2_poly.max_rel_error(fitted) < 1.5e-4
 
 
 def test_emulated_device_function_error():
@@ -52,11 +53,13 @@ def test_emulated_device_function_error():
     y = np.array([emulate(v) for v in x[::7]] + [emulate(v) for v in x[-300:]], np.float64)
     xs = np.concatenate([x[::7], x[-300:]]).astype(np.float64)
     rel = np.abs(y - np.exp2(xs)) / np.exp2(xs)
-    assert rel.max() < 1e-4, rel.max()
+    assert rel.max() < 1.5e-4, rel.max()
 
 
 def test_masked_scores_vanish():
     for x in (-np.inf, -1e30, -127.0, -200.0):
         y = float(emulate(np.float32(x)))
         assert 0.0 <= y <= 2.0 ** -125
-    assert abs(float(emulate(np.float32(0.0))) - 1.0) < 1e-4
+    assert float(emulate(np.float32(0.0))) == 1.0   # a row's largest score: P = 1 exactly
+    for j in range(-20, 8):
+        assert float(emulate(np.float32(j))) == 2.0 ** j

@@ -82,7 +82,7 @@ def attended_max(q, k, v, scale, causal, lse, top=32, chunk=1024):
     return out
 
 
-def check_against_emulation(o, lse, o_emu, lse_emu, q, k, v, causal, scale, sigma=None):
+def check_against_emulation(o, lse, o_emu, lse_emu, q, k, v, causal, scale, sigma=None, single_tile=None):
     exact, lse_exact = oracle.attention_forward(q, k, v, causal, scale)
     M = attended_max(q, k, v, scale, causal, lse_exact)
     bound = O_MAX_ABS + 0.25 * M
@@ -98,7 +98,10 @@ def check_against_emulation(o, lse, o_emu, lse_emu, q, k, v, causal, scale, sigm
     rms_gpu = math.sqrt(np.mean((o - exact) ** 2))
     assert rms_diff <= FP8_RMS_RATIO * rms_emu, (rms_diff, rms_emu)
     assert rms_gpu <= 1.1 * rms_emu + 1e-4, (rms_gpu, rms_emu)
-    o_one, _ = oracle.fp8_attention_forward(q, k, v, causal, scale, sigma, tile=1 << 30)
+    if single_tile is None:
+        o_one, _ = oracle.fp8_attention_forward(q, k, v, causal, scale, sigma, tile=1 << 30)
+    else:
+        o_one = single_tile()
     rms_one = math.sqrt(np.mean((o_one - exact) ** 2))
     assert rms_gpu <= 1.1 * rms_one + 1e-4, (rms_gpu, rms_one)
     return exact
