@@ -12,7 +12,8 @@ larger than the 126 MB L2, so no flush runs between steps.
 The JSON line also carries: `e2e`, the same step through the public API with
 every step's inputs copied from pinned host memory and all results read back
 (three streams, two buffer sets: neighbouring steps' copies overlap the
-kernels); `fp8`, the FP8 workload's pre-pass + forward in TFLOP/s; `decode`,
+kernels); `fp8`, the FP8 workload's pre-pass + forward in TFLOP/s (and the
+MXFP8 forward on the same inputs); `decode`,
 one decode step (a query row per head against a 16K-key cache) in GB/s against
 the measured HBM copy bandwidth.
 
@@ -577,19 +578,39 @@ def run_fp8_leg(args, fa, stream):
         b_.record(stream)
     torch.cuda.synchronize()
     ms_k = statistics.mean(a.elapsed_time(b_) for a, b_ in ev)
+    # the MXFP8 forward (32-element E8M0 block scales applied by the tensor
+    # cores; pre-pass + forward in one call), same inputs
+    ws_mx = torch.empty(fa.fa_mxfp8_workspace_size(w.B, w.Hq, w.Hkv, w.N, w.d), dtype=torch.uint8, device="cuda")
+
+    def call_mx():
+        fa.fa_fwd_mxfp8(dev["q"], dev["k"], dev["v"], causal=causal, rotation_seed=w.seed, use_rotation=True,
+                        scale_rule="fit", out=o, lse=lse, workspace=ws_mx)
+
+    for _ in range(args.warmup):
+        call_mx()
+    torch.cuda.synchronize()
+    for a, b_ in ev:
+        a.record(stream)
+        call_mx()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    ms_mx = statistics.mean(a.elapsed_time(b_) for a, b_ in ev)
     pk, pk_kind = peaks()
-    bf16_peak, which = choose_peak(pk, steps * (ms + ms_k), None)
+    bf16_peak, which = choose_peak(pk, steps * (ms + ms_k + ms_mx), None)
     fp8_peak = 2.0 * bf16_peak
     tf = w.fwd_flops(causal) / (ms * 1e-3) / 1e12
     tf_k = w.fwd_flops(causal) / (ms_k * 1e-3) / 1e12
+    tf_mx = w.fwd_flops(causal) / (ms_mx * 1e-3) / 1e12
     return {"workload": f"fp8: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} causal={causal} e4m3",
             "tflops": tf, "ms_per_call": ms, "calls": steps,
             "kernel_only_tflops": tf_k, "kernel_only_ms": ms_k,
             "peak": fp8_peak, "peak_kind": f"nominal: {pk_kind} bf16 dense {which} x 2 (the datasheet's fp8:bf16 "
                                               "ratio; no fp8 peak is measured)",
             "frac_of_peak": tf / fp8_peak, "kernel_only_frac_of_peak": tf_k / fp8_peak,
+            "mxfp8_tflops": tf_mx, "mxfp8_ms_per_call": ms_mx, "mxfp8_frac_of_peak": tf_mx / fp8_peak,
             "includes": "tflops: quantisation pre-pass (Hadamard rotation, 64-row block scales) + FP8 forward; "
-                        "kernel_only: the FP8 forward from an already quantised workspace"}
+                        "kernel_only: the FP8 forward from an already quantised workspace; "
+                        "mxfp8: fa_fwd_mxfp8 (rule fit: MX pre-pass + MXFP8 forward)"}
 
 
 def run_decode_leg(args, fa, stream):

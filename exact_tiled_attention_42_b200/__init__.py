@@ -16,12 +16,14 @@ from .api import (  # noqa: F401
     fa_bwd_varlen,
     fa_bwd_varlen_workspace_size,
     fa_fwd_fp8,
+    fa_fwd_mxfp8,
     fa_fp8_quantize,
     fa_fwd_fp8_quantized,
     fa_fwd_decode,
     fa_decode_workspace_size,
     fa_bwd_workspace_size,
     fa_fp8_workspace_size,
+    fa_mxfp8_workspace_size,
     fa_status_string,
     fa_last_device_status,
 )

@@ -26,6 +26,9 @@ SIGNATURES = {
     "fa_fp8_workspace_size": (_c_size_t, [_c_int] * 5),
     "fa_fwd_fp8": (_c_int, [_c_void_p] * 5 + [_c_uint64, _c_int, _c_void_p, _c_size_t] + [_c_int] * 6
                    + [_c_float, _c_void_p]),
+    "fa_mxfp8_workspace_size": (_c_size_t, [_c_int] * 5),
+    "fa_fwd_mxfp8": (_c_int, [_c_void_p] * 5 + [_c_uint64, _c_int, _c_int, _c_void_p, _c_size_t] + [_c_int] * 6
+                     + [_c_float, _c_void_p]),
     "fa_decode_workspace_size": (_c_size_t, [_c_int] * 7),
     "fa_fp8_quantize": (_c_int, [_c_void_p] * 3 + [_c_uint64, _c_int, _c_void_p, _c_size_t] + [_c_int] * 5 + [_c_void_p]),
     "fa_fwd_fp8_quantized": (_c_int, [_c_void_p, _c_size_t, _c_void_p, _c_void_p] + [_c_int] * 7 + [_c_float, _c_void_p]),

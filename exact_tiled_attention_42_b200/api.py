@@ -162,6 +162,42 @@ def fa_fwd_fp8(q, k, v, causal: bool = False, scale: float | None = None, rotati
     return out, lse
 
 
+def fa_mxfp8_workspace_size(B: int, Hq: int, Hkv: int, N: int, d: int) -> int:
+    return int(_lib.load().fa_mxfp8_workspace_size(B, Hq, Hkv, N, d))
+
+
+MX_SCALE_RULES = {"ocp": 0, "fit": 1}
+
+
+def fa_fwd_mxfp8(q, k, v, causal: bool = False, scale: float | None = None, rotation_seed: int = 0,
+                 use_rotation: bool = True, scale_rule: str = "fit", out=None, lse=None, workspace=None,
+                 stream=None):
+    """MXFP8 forward (e4m3 with one E8M0 exponent per 32 elements along each
+    product's contraction, applied by the tensor cores); bf16 inputs and
+    output, d = 128. scale_rule "ocp" (the MX specification's exponent) or
+    "fit" (one higher where that would saturate)."""
+    B, Hq, Hkv, N, d = _dims(q, k)
+    _check("q", q, torch.bfloat16, (B, Hq, N, d))
+    _check("k", k, torch.bfloat16, (B, Hkv, N, d))
+    _check("v", v, torch.bfloat16, (B, Hkv, N, d))
+    if scale_rule not in MX_SCALE_RULES:
+        raise ValueError(f"scale_rule must be one of {sorted(MX_SCALE_RULES)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    if workspace is None:
+        workspace = torch.empty(fa_mxfp8_workspace_size(B, Hq, Hkv, N, d), dtype=torch.uint8, device=q.device)
+    st = _lib.load().fa_fwd_mxfp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                  int(rotation_seed) & 0xFFFFFFFFFFFFFFFF, int(bool(use_rotation)),
+                                  MX_SCALE_RULES[scale_rule], workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(),
+                                  B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream(stream))
+    if st != FA_OK:
+        raise FAError("fa_fwd_mxfp8", st)
+    return out, lse
+
+
 def fa_fp8_quantize(q, k, v, rotation_seed: int = 0, use_rotation: bool = True, workspace=None, stream=None):
     """The FP8 pre-pass alone: rotated (optional) and 64-row block-quantised
     e4m3 copies of q, k, v with their scales, in a workspace (uint8 tensor)

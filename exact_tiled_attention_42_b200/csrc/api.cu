@@ -571,3 +571,85 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
 }
 
 }  // extern "C"
+
+namespace {
+
+// MXFP8 workspace: e4m3 codes of Q, K, V, then the exponent bytes of Q, K
+// (4 per row) and V (nb32p per column), each region 1024-byte aligned.
+struct MxLayout {
+  size_t cq, ckv, eq, ekv, ev;
+  int nb32p;
+};
+MxLayout mx_layout(int B, int Hq, int Hkv, int N, int d) {
+  MxLayout L;
+  L.nb32p = 4 * ((N + 127) / 128);
+  const size_t q = static_cast<size_t>(B) * Hq, kv = static_cast<size_t>(B) * Hkv;
+  L.cq = up1024(q * N * d);
+  L.ckv = up1024(kv * N * d);
+  L.eq = up1024(q * N * 4);
+  L.ekv = up1024(kv * N * 4);
+  L.ev = up1024(kv * d * L.nb32p);
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa_mxfp8_workspace_size(int B, int Hq, int Hkv, int N, int d) {
+  if (check_shape(B, Hq, Hkv, N, d, 1.0f) != FA_OK || d != 128) return 0;
+  const MxLayout L = mx_layout(B, Hq, Hkv, N, d);
+  return L.cq + 2 * L.ckv + L.eq + L.ekv + L.ev;
+}
+
+fa_status fa_fwd_mxfp8(const void* q, const void* k, const void* v, void* o, float* lse, uint64_t rotation_seed,
+                       int use_rotation, int scale_rule, void* workspace, size_t workspace_bytes, int B, int Hq,
+                       int Hkv, int N, int d, int causal, float scale, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  fa_status st = check_shape(B, Hq, Hkv, N, d, scale);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;  // built for d = 128
+  if (scale_rule != 0 && scale_rule != 1) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < fa_mxfp8_workspace_size(B, Hq, Hkv, N, d)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  const long long BH = static_cast<long long>(B) * Hq, BHkv = static_cast<long long>(B) * Hkv;
+  if (BH > 65535) return FA_ERR_UNSUPPORTED;  // pre-pass grid.y
+  const MxLayout L = mx_layout(B, Hq, Hkv, N, d);
+  char* ws = static_cast<char*>(workspace);
+  fa::MxParams p;
+  p.src[0] = static_cast<const uint16_t*>(q);
+  p.src[1] = static_cast<const uint16_t*>(k);
+  p.src[2] = static_cast<const uint16_t*>(v);
+  p.codes[0] = reinterpret_cast<uint8_t*>(ws);
+  p.codes[1] = reinterpret_cast<uint8_t*>(ws + L.cq);
+  p.codes[2] = reinterpret_cast<uint8_t*>(ws + L.cq + L.ckv);
+  p.exps[0] = reinterpret_cast<uint8_t*>(ws + L.cq + 2 * L.ckv);
+  p.exps[1] = reinterpret_cast<uint8_t*>(ws + L.cq + 2 * L.ckv + L.eq);
+  p.exps[2] = reinterpret_cast<uint8_t*>(ws + L.cq + 2 * L.ckv + L.eq + L.ekv);
+  p.heads[0] = static_cast<int>(BH);
+  p.heads[1] = static_cast<int>(BHkv);
+  p.heads[2] = static_cast<int>(BHkv);
+  p.rotation_seed = rotation_seed;
+  p.rotate = use_rotation != 0;
+  p.fit = scale_rule;
+  p.lse = lse;
+  p.status = status_ptr();
+  p.N = N;
+  p.nb32p = L.nb32p;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.num_qtiles = (N + 127) / 128;
+  p.score_log2 = scale * 1.4426950408889634f / (p.rotate ? static_cast<float>(d) : 1.0f);
+  if (!p.status) return FA_ERR_CUDA;
+  CUtensorMap tmQ, tmK, tmV, tmO;
+  if (!make_map_e4m3(&tmQ, p.codes[0], d, N, BH) || !make_map_e4m3(&tmK, p.codes[1], d, N, BHkv) ||
+      !make_map_e4m3(&tmV, p.codes[2], d, N, BHkv) || !make_map_bf16(&tmO, o, d, N, BH, 128))
+    return FA_ERR_CUDA;
+  if (fa::launch_mxfp8_quant(p, stream) != cudaSuccess) return FA_ERR_CUDA;
+  cudaError_t e = fa::launch_fwd_mxfp8(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), causal != 0, stream);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -110,6 +110,36 @@ cudaError_t launch_fp8_quant(const Fp8Params& p, cudaStream_t stream);
 cudaError_t launch_fwd_fp8(const CUtensorMap& tmQ8, const CUtensorMap& tmK8, const CUtensorMap& tmV8,
                            const CUtensorMap& tmO, const Fp8Params& p, int BH, bool causal, cudaStream_t stream);
 
+struct MxParams {
+  // pre-pass
+  const uint16_t* src[3];  // bf16 Q [B*Hq, N, d], K and V [B*Hkv, N, d]
+  uint8_t* codes[3];       // e4m3 copies (Q and K rotated when rotate != 0), same layouts
+  uint8_t* exps[3];        // E8M0 exponents (e + 127): Q [B*Hq, N, 4] and K [B*Hkv, N, 4] (one per
+                           // 32 columns), V [B*Hkv, d, nb32p] (one per 32 keys of a column)
+  int heads[3];            // B*Hq, B*Hkv, B*Hkv
+  uint64_t rotation_seed;
+  int rotate;
+  int fit;                 // 1: exponent one higher when amax's significand exceeds 1.75
+  // forward
+  float* lse;              // [B*Hq, N]
+  int* status;
+  int N;
+  int nb32p;               // 4 * ceil(N / 128): V's 32-key blocks per column, whole 128-key tiles
+  int Hq;
+  int Hkv;
+  int group;
+  int num_qtiles;
+  float score_log2;        // scale * log2(e), divided by d when rotated
+};
+
+// MXFP8 pre-pass (rotation + MX quantisation of Q, K along d and of V along
+// the keys) and the MXFP8 forward (d = 128; one query tile per CTA, grid
+// BH * p.num_qtiles). tmQ8/tmK8/tmV8: e4m3 [B*H, N, d], 128 x 128 boxes, 128B
+// swizzle; tmO: bf16 output map as for the bf16 forward.
+cudaError_t launch_mxfp8_quant(const MxParams& p, cudaStream_t stream);
+cudaError_t launch_fwd_mxfp8(const CUtensorMap& tmQ8, const CUtensorMap& tmK8, const CUtensorMap& tmV8,
+                             const CUtensorMap& tmO, const MxParams& p, int BH, bool causal, cudaStream_t stream);
+
 struct DecParams {
   const uint16_t* q;  // bf16 [B*Hq, Nq, d]
   uint16_t* o;        // bf16 [B*Hq, Nq, d]

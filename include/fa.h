@@ -223,6 +223,45 @@ fa_status fa_fwd_fp8_quantized(const void* workspace, size_t workspace_bytes, vo
                                float scale, cudaStream_t stream);
 
 /*
+ * Bytes of device workspace fa_fwd_mxfp8 needs: e4m3 codes of Q, K, V and
+ * their E8M0 exponent bytes (layout at fa_fwd_mxfp8). Returns 0 for invalid
+ * sizes and for d != 128.
+ */
+size_t fa_mxfp8_workspace_size(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * MXFP8 forward: the FP8 forward with the block quantisation that B200's
+ * tensor cores apply in hardware. "FlashAttention-3: Fast and Accurate
+ * Attention with Asynchrony and Low-precision" (abstract) names block
+ * quantisation without fixing the block; here each block is 32 elements
+ * along a product's contraction with one power-of-two (E8M0) scale, per the
+ * OCP Microscaling Formats (MX) specification v1.0:
+ *   Q and K (after the rotation diag(sigma) H_d when use_rotation != 0, as in
+ *   fa_fwd_fp8): each row in blocks of 32 columns;
+ *   V: each column in blocks of 32 keys;
+ *   P: each row of each 128-key tile in blocks of 32 keys.
+ * Shared exponent e = floor(log2 amax) - 8 clamped to [-127, 127] (-127 for
+ * a zero block), codes e4m3(x 2^-e) with saturation at 448 (scale_rule 0,
+ * the specification's); scale_rule 1 takes e + 1 where amax's significand
+ * exceeds 1.75, so that no element saturates. Other scale_rule values:
+ * FA_ERR_INVALID_ARG. Only d = 128 is built (FA_ERR_UNSUPPORTED otherwise);
+ * B * Hq at most 65535. bf16 q [B, Hq, N, d], k, v [B, Hkv, N, d] and o
+ * [B, Hq, N, d], float32 lse [B, Hq, N], all 16-byte aligned and owned by the
+ * caller. The workspace (at least fa_mxfp8_workspace_size bytes, 16-byte
+ * aligned, else FA_ERR_WORKSPACE / FA_ERR_MISALIGNED) is overwritten; it then
+ * holds, each region starting on a 1024-byte boundary: e4m3 codes of Q
+ * [B*Hq, N, d], K and V [B*Hkv, N, d]; exponent bytes (e + 127) of Q
+ * [B*Hq, N, 4] and K [B*Hkv, N, 4] (one per 32 columns), and of V
+ * [B*Hkv, d, nb] with nb = 4 * ceil(N / 128) (one per 32 keys of a column;
+ * blocks past N hold the exponent of zeros, 0).
+ */
+fa_status fa_fwd_mxfp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                       uint64_t rotation_seed, int use_rotation, int scale_rule,
+                       void* workspace, size_t workspace_bytes,
+                       int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                       cudaStream_t stream);
+
+/*
  * Bytes of device workspace fa_fwd_decode needs for these sizes and
  * num_ctas (0 = automatic, as in fa_fwd_decode): for each CTA of the split
  * pass and each KV head, a float32 partial output row and a float32

@@ -30,7 +30,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for need in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_fwd_fp8", "fa_fp8_workspace_size",
-                 "fa_status_string", "fa_last_device_status"):
+                 "fa_fwd_mxfp8", "fa_mxfp8_workspace_size", "fa_status_string", "fa_last_device_status"):
         assert need in names
 
 
@@ -153,6 +153,25 @@ def test_fp8_rejects_bad_arguments(lib):
     assert lib.fa_fwd_fp8_quantized(P, ws, None, P, 1, 1, 2, 2, 128, 128, 0, 0.1, None) == 1
     assert lib.fa_fwd_fp8_quantized(P, ws, P + 2, P, 1, 1, 2, 2, 128, 128, 0, 0.1, None) == 3
     assert lib.fa_fwd_fp8_quantized(P, ws, P, P, 1, 1, 3, 2, 128, 128, 0, 0.1, None) == 1  # Hq % Hkv
+
+
+def test_mxfp8_rejects_bad_arguments(lib):
+    ws = lib.fa_mxfp8_workspace_size(1, 2, 2, 300, 128)
+    # codes 2*300*128 each (three regions), exponents Q and K 2*300*4 each, V 2*128*12
+    up = lambda x: (x + 1023) // 1024 * 1024
+    assert ws == 3 * up(2 * 300 * 128) + 2 * up(2 * 300 * 4) + up(2 * 128 * 12)
+    assert lib.fa_mxfp8_workspace_size(1, 2, 2, 300, 64) == 0                 # d = 128 only
+    def mx(q=P, rule=1, wsp=P, wsb=ws, Hq=2, d=128):
+        return lib.fa_fwd_mxfp8(q, P, P, P, P, 7, 1, rule, wsp, wsb, 1, Hq, 2, 300, d, 0, 0.1, None)
+    assert mx(q=None) == 1
+    assert mx(d=64) == 2
+    assert mx(rule=2) == 1
+    assert mx(rule=-1) == 1
+    assert mx(q=P + 8) == 3
+    assert mx(wsp=None) == 4
+    assert mx(wsb=ws - 1) == 4
+    assert mx(wsp=P + 4) == 3
+    assert mx(Hq=3) == 1                                                      # Hq % Hkv
 
 
 def test_workspace_sizes_are_linear_in_n(lib):
