@@ -218,6 +218,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.group = Hq / Hkv;
   p.num_qtiles = (N + 127) / 128;
   p.num_pairs = (p.num_qtiles + 1) / 2;
+  p.raster_heads = fa::raster_heads_for(BH, Hq / Hkv, 4ll * N * d);
   p.scale_log2 = scale * 1.4426950408889634f;
 #ifdef FA_DEBUG_WITHHOLD
   p.debug_withhold = g_debug_withhold;
@@ -260,6 +261,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   p.group = Hq / Hkv;
   p.num_qtiles = (max_seqlen + 127) / 128;
   p.num_pairs = (p.num_qtiles + 1) / 2;
+  p.raster_heads = fa::raster_heads_for(static_cast<long long>(B) * Hq, Hq / Hkv, 4ll * max_seqlen * d);
   p.scale_log2 = scale * 1.4426950408889634f;
 #ifdef FA_DEBUG_WITHHOLD
   p.debug_withhold = 0;
@@ -501,6 +503,7 @@ fa_status fp8_setup(fa::Fp8Params* p, void* workspace, size_t workspace_bytes, i
   p->group = Hq / Hkv;
   p->num_qtiles = (N + 127) / 128;
   p->num_pairs = (p->num_qtiles + 1) / 2;
+  p->raster_heads = fa::raster_heads_for(BH, Hq / Hkv, 2ll * N * d);  // e4m3 K and V
   p->score_log2 = scale * 1.4426950408889634f / (p->rotate ? static_cast<float>(d) : 1.0f);
   p->status = nullptr;  // set by the caller once every argument has been checked
   return FA_OK;

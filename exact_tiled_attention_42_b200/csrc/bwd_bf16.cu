@@ -342,13 +342,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         constexpr uint32_t IDESC_TS = idesc_bf16(BT, D, false, true);
         constexpr uint32_t IDESC_DQ = idesc_bf16(BT, D, true, true);
         const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
+        // K and V stay put for the whole CTA: their descriptors are fixed
+        const uint64_t dk_ss = smem_desc_sw128(sK, 16, 1024), dv_ss = smem_desc_sw128(sV, 16, 1024);
+        const uint64_t dk_mn = smem_desc_sw128(sK, C::BOX_BYTES, 1024);
         auto issue_st = [&](int it) {  // S^T = K_j Q_i^T into the S^T columns
-          const uint32_t sQ = base + C::OFF_Q + (it & 1) * C::TILE_BYTES;
+          const uint64_t dq = smem_desc_sw128(base + C::OFF_Q + (it & 1) * C::TILE_BYTES, 16, 1024);
   #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-            mma_ss(tmem + C::COL_S, smem_desc_sw128(sK + off, 16, 1024), smem_desc_sw128(sQ + off, 16, 1024),
-                   IDESC_SS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_S, desc_plus(dk_ss, off), desc_plus(dq, off), IDESC_SS, kk > 0 ? 1u : 0u);
           }
           mma_commit(bars.s_full());
         };
@@ -371,19 +373,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           if (C::DQ_SHARES_DP && it > 0 && !mbar_wait_sleep(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
             break;
           tc_fence_after();
+          const uint64_t ddo = smem_desc_sw128(sdO, 16, 1024), ddo_mn = smem_desc_sw128(sdO, C::BOX_BYTES, 1024);
+          const uint64_t dq_mn = smem_desc_sw128(sQ, C::BOX_BYTES, 1024);
   #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V_j dO_i^T
             const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-            mma_ss(tmem + C::COL_DP, smem_desc_sw128(sV + off, 16, 1024), smem_desc_sw128(sdO + off, 16, 1024),
-                   IDESC_SS, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_DP, desc_plus(dv_ss, off), desc_plus(ddo, off), IDESC_SS, kk > 0 ? 1u : 0u);
           }
           mma_commit(bars.dp_full());
           if (!mbar_wait_sleep(bars.p_ready(), it & 1, abort, p.status, SITE_BWD + 7)) break;
           tc_fence_after();
   #pragma unroll
           for (int kk = 0; kk < BT / 16; ++kk)  // dV += P^T dO_i
-            mma_ts(tmem + C::COL_DV, tmem + C::COL_S + (kk >> 2) * 64 + (kk & 3) * 8,
-                   smem_desc_sw128(sdO + kk * 2048, C::BOX_BYTES, 1024),
+            mma_ts(tmem + C::COL_DV, tmem + C::COL_S + (kk >> 2) * 64 + (kk & 3) * 8, desc_plus(ddo_mn, kk * 2048),
                    IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bars.dv_done());
           if (it + 1 < n_it) {
@@ -395,8 +397,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           tc_fence_after();
   #pragma unroll
           for (int kk = 0; kk < BT / 16; ++kk)  // dK += dS^T Q_i (dS^T over the dP^T columns)
-            mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + (kk >> 2) * 64 + (kk & 3) * 8,
-                   smem_desc_sw128(sQ + kk * 2048, C::BOX_BYTES, 1024),
+            mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + (kk >> 2) * 64 + (kk & 3) * 8, desc_plus(dq_mn, kk * 2048),
                    IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bars.q_empty(st));
           if (!mbar_wait_sleep(bars.dss_ready(), it & 1, abort, p.status, SITE_BWD + 16)) break;
@@ -404,11 +405,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
               !mbar_wait_sleep(bars.dq_free(), (it - 1) & 1, abort, p.status, SITE_BWD + 6))
             break;
           tc_fence_after();
-          const uint32_t sdS = ds_smem(st);
+          const uint64_t dds = smem_desc_sw128(ds_smem(st), 16384, 1024);
   #pragma unroll
           for (int kk = 0; kk < BT / 16; ++kk)  // dQ_i = dS K_j (A and B MN-major)
-            mma_ss(tmem + C::COL_DQ, smem_desc_sw128(sdS + kk * 2048, 16384, 1024),
-                   smem_desc_sw128(sK + kk * 2048, C::BOX_BYTES, 1024), IDESC_DQ, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_DQ, desc_plus(dds, kk * 2048), desc_plus(dk_mn, kk * 2048), IDESC_DQ,
+                   kk > 0 ? 1u : 0u);
           mma_commit(bars.dq_full());
           mma_commit(bars.do_empty(st));
         }

@@ -113,12 +113,11 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // 1-D grid: heads vary fastest and the query-tile pairs with the most key
-  // tiles (causal) come first across all heads, so the light pairs form the
-  // tail (measured faster than running each head's pairs back to back).
+  // 1-D grid in groups of heads (raster_pairs): inside a group the pairs with
+  // the most key tiles (causal) come first, heads fastest.
   const int BH = static_cast<int>(gridDim.x) / p.num_pairs;
-  const int bh = static_cast<int>(blockIdx.x) % BH;  // b * Hq + hq
-  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
+  int bh, pair;  // bh = b * Hq + hq
+  raster_pairs(static_cast<int>(blockIdx.x), BH, p.num_pairs, p.raster_heads, bh, pair);
   const int b = bh / p.Hq;
   const int hq = bh - b * p.Hq;
   // A packed batch's sequence b: tokens s0 .. s0 + len - 1 (its own N). CTAs
@@ -249,24 +248,22 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         const uint32_t sQ = base + C::OFF_Q;
         auto issue_qk = [&](int x, int stage) {
           const uint32_t dS = tmem + (x ? C::COL_S1 : C::COL_S0);
-          const uint32_t qa = sQ + x * C::TILE_BYTES;
-          const uint32_t kb = base + C::OFF_K + stage * C::TILE_BYTES;
+          const uint64_t da = smem_desc_sw128(sQ + x * C::TILE_BYTES, 16, 1024);
+          const uint64_t db = smem_desc_sw128(base + C::OFF_K + stage * C::TILE_BYTES, 16, 1024);
   #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-            mma_ss(dS, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), IDESC_QK,
-                   kk > 0 ? 1u : 0u);
+            mma_ss(dS, desc_plus(da, off), desc_plus(db, off), IDESC_QK, kk > 0 ? 1u : 0u);
           }
         };
         auto issue_pv = [&](int x, int stage, bool accumulate) {
           const uint32_t dO = tmem + (x ? C::COL_O1 : C::COL_O0);
           const uint32_t aP = tmem + (x ? C::COL_S1 : C::COL_S0);
-          const uint32_t vb = base + C::OFF_V + stage * C::TILE_BYTES;
+          const uint64_t dv = smem_desc_sw128(base + C::OFF_V + stage * C::TILE_BYTES, C::BOX_BYTES, 1024);
   #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             // 16 keys = two 8-row groups of the MN-major V tile; 16 bf16 of P = 8 columns.
-            mma_ts(dO, aP + kk * 8, smem_desc_sw128(vb + kk * 16 * 128, C::BOX_BYTES, 1024), IDESC_PV,
-                   (accumulate || kk > 0) ? 1u : 0u);
+            mma_ts(dO, aP + kk * 8, desc_plus(dv, kk * 16 * 128), IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
           }
         };
         bool ok = mbar_wait_sleep(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&

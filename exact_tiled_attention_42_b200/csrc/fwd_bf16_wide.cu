@@ -206,11 +206,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int s = j % C::NS;
         if (!mbar_wait_sleep(bars.k_full(s), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) return false;
         tc_fence_after();
-        const uint32_t kb = base + C::OFF_K + s * C::KV_BYTES;
+        const uint64_t da = smem_desc_sw128(sQ, 16, 1024);
+        const uint64_t db = smem_desc_sw128(base + C::OFF_K + s * C::KV_BYTES, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::COL_S + (j & 1) * 64, smem_desc_sw128(sQ + (kk >> 2) * C::QBOX + (kk & 3) * 32, 16, 1024),
-                 smem_desc_sw128(kb + (kk >> 2) * C::KBOX + (kk & 3) * 32, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + C::COL_S + (j & 1) * 64, desc_plus(da, (kk >> 2) * C::QBOX + (kk & 3) * 32),
+                 desc_plus(db, (kk >> 2) * C::KBOX + (kk & 3) * 32), IDESC_QK, kk > 0 ? 1u : 0u);
         mma_commit(bars.s_full(j & 1));
         mma_commit(bars.k_empty(s));
         return true;
@@ -223,13 +224,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait_sleep(bars.v_full(s), (j / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
         if (!mbar_wait_sleep(bars.p_full(j & 1), (j >> 1) & 1, abort, p.status, SITE_P_FULL)) break;
         tc_fence_after();
-        const uint32_t vb = base + C::OFF_V + s * C::KV_BYTES;
+        const uint64_t dv = smem_desc_sw128(base + C::OFF_V + s * C::KV_BYTES, C::KBOX, 1024);
         // O += P_j V_j: 16 keys per instruction (P: 8 columns of bf16 pairs;
         // V: two 8-row groups of the MN-major 64-row tile)
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + C::COL_O, tmem + C::COL_S + (j & 1) * 64 + kk * 8,
-                 smem_desc_sw128(vb + kk * 16 * 128, C::KBOX, 1024), IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + C::COL_O, tmem + C::COL_S + (j & 1) * 64 + kk * 8, desc_plus(dv, kk * 16 * 128), IDESC_PV,
+                 (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bars.v_empty(s));
         mma_commit(bars.pv_done());
         if (j + 2 < nkv && !issue_s(j + 2)) break;

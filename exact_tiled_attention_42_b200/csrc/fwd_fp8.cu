@@ -14,7 +14,10 @@
 //        scales; the 256 keeps small probabilities above e4m3's subnormals)
 //   O = (sum P~ Vc) * max sV / 256 / l,   l = sum of unquantised P.
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512); P~ (4 e4m3 per
-// column) over the first 32 columns of its S.
+// column) over the first 32 columns of its S. The next S_x is issued in two
+// parts: the keys over columns 32-127 as soon as the softmax has read S_x into
+// registers (s_free), overlapping that softmax; the keys over P's columns
+// after P V has read P.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -23,6 +26,9 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BN = 128;
+// P overwrites the first P_COLS score columns of its tile (e4m3, four keys per
+// 32-bit column), so only the keys of those columns wait for P V to have read P.
+constexpr int P_COLS = BN / 4;
 constexpr int D = 128;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
@@ -46,9 +52,10 @@ static_assert(P_LIFT * 1.7411011f <= 448.f, "2^TAU * P_LIFT must stay within e4m
 // Of every 8 groups of 4 scores, this many take their exponentials on the FMA
 // pipe (exp2_poly) instead of MUFU: the two query tiles' 2 x 128 x 128
 // exponentials per key tile need 2048 MUFU cycles against about 1080 of e4m3
-// MMA. Measured on the FP8 workload (forward alone): 0 -> 1205, 2 -> 1279,
-// 3 -> 1186 TFLOP/s.
-constexpr int POLY_GROUPS = 2;
+// MMA, but the polynomial costs issue slots the softmax also needs. Measured
+// on the FP8 workload (forward alone, next S split around P's columns):
+// 0 -> 1223, 1 -> 1223, 2 -> 1195, 3 -> 1113 TFLOP/s.
+constexpr int POLY_GROUPS = 1;
 
 // exp2_poly on two values with packed FMA-pipe arithmetic.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
@@ -64,7 +71,7 @@ struct Cfg {
   static constexpr int OFF_O = OFF_V + NS * TILE_BYTES;  // bf16 output staging, 2 x 32 KB
   static constexpr int O_TILE_BYTES = BM * D * 2;
   static constexpr int OFF_BAR = OFF_O + 2 * O_TILE_BYTES;
-  static constexpr int NUM_BARS = 1 + 4 * NS + 9;
+  static constexpr int NUM_BARS = 1 + 4 * NS + 11;
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 384;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -83,6 +90,9 @@ struct Bars {
   __device__ uint32_t o_done(int x) const { return base + 8u * (5 + 4 * Cfg::NS + x); }
   __device__ uint32_t teardown() const { return base + 8u * (7 + 4 * Cfg::NS); }
   __device__ uint32_t epi(int x) const { return base + 8u * (8 + 4 * Cfg::NS + x); }
+  // the softmax of query tile x has read S_x into registers: the score
+  // columns past P's may take the next tile's S
+  __device__ uint32_t s_free(int x) const { return base + 8u * (10 + 4 * Cfg::NS + x); }
 };
 
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -122,12 +132,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // 1-D grid: heads vary fastest and the query-tile pairs with the most key
-  // tiles (causal) come first across all heads, so the light pairs form the
-  // tail (measured faster than running each head's pairs back to back).
+  // 1-D grid in groups of heads (raster_pairs): inside a group the pairs with
+  // the most key tiles (causal) come first, heads fastest.
   const int BH = static_cast<int>(gridDim.x) / p.num_pairs;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
+  int bh, pair;
+  raster_pairs(static_cast<int>(blockIdx.x), BH, p.num_pairs, p.raster_heads, bh, pair);
   const int b = bh / p.Hq;
   const int hq = bh - b * p.Hq;
   const int kvh = b * p.Hkv + hq / p.group;
@@ -154,6 +163,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bars.p_full(x), 4);
       mbar_init(bars.o_done(x), 1);
       mbar_init(bars.epi(x), 4);
+      mbar_init(bars.s_free(x), 4);
     }
     mbar_init(bars.teardown(), 1);
     *abort = 0;
@@ -209,34 +219,37 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == MMA_WARP) {
       if (lane == 0) {
         constexpr uint32_t IDESC_QK = idesc_e4m3(BM, BN, false, false);
+        constexpr uint32_t IDESC_QK_HEAD = idesc_e4m3(BM, P_COLS, false, false);
+        constexpr uint32_t IDESC_QK_TAIL = idesc_e4m3(BM, BN - P_COLS, false, false);
         constexpr uint32_t IDESC_PV = idesc_e4m3(BM, D, false, true);
         const uint32_t sQ = base + C::OFF_Q;
-        auto issue_qk = [&](int x, int stage) {
-          const uint32_t dS = tmem + (x ? C::COL_S1 : C::COL_S0);
-          const uint32_t qa = sQ + x * C::TILE_BYTES;
-          const uint32_t kb = base + C::OFF_K + stage * C::TILE_BYTES;
+        // S_x = Q_x K^T over keys [key0, key0 + N) of the stage, into the
+        // score columns of those keys (128-byte K rows: key0 * 128 bytes is a
+        // whole number of 8-row swizzle atoms)
+        auto issue_qk = [&](int x, int stage, int key0, uint32_t idesc) {
+          const uint32_t dS = tmem + (x ? C::COL_S1 : C::COL_S0) + key0;
+          const uint64_t da = smem_desc_sw128(sQ + x * C::TILE_BYTES, 16, 1024);
+          const uint64_t db = smem_desc_sw128(base + C::OFF_K + stage * C::TILE_BYTES + key0 * 128, 16, 1024);
   #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)  // 32 e4m3 = 32 bytes of each 128-byte row
-            mma_ss_f8(dS, smem_desc_sw128(qa + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 32, 16, 1024), IDESC_QK,
-                      kk > 0 ? 1u : 0u);
+            mma_ss_f8(dS, desc_plus(da, kk * 32), desc_plus(db, kk * 32), idesc, kk > 0 ? 1u : 0u);
         };
         auto issue_pv = [&](int x, int stage, bool accumulate) {
           const uint32_t dO = tmem + (x ? C::COL_O1 : C::COL_O0);
           const uint32_t aP = tmem + (x ? C::COL_S1 : C::COL_S0);
-          const uint32_t vb = base + C::OFF_V + stage * C::TILE_BYTES;
+          const uint64_t dv = smem_desc_sw128(base + C::OFF_V + stage * C::TILE_BYTES, 16384, 1024);
   #pragma unroll
           for (int kk = 0; kk < BN / 32; ++kk)  // 32 keys = four 8-row groups; 32 e4m3 of P = 8 columns
-            mma_ts_f8(dO, aP + kk * 8, smem_desc_sw128(vb + kk * 4096, 16384, 1024), IDESC_PV,
-                      (accumulate || kk > 0) ? 1u : 0u);
+            mma_ts_f8(dO, aP + kk * 8, desc_plus(dv, kk * 4096), IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
         };
         bool ok = mbar_wait_sleep(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&
                   mbar_wait_sleep(bars.k_full(0), 0, abort, p.status, SITE_K_FULL);
         if (ok) {
           tc_fence_after();
-          issue_qk(0, 0);
+          issue_qk(0, 0, 0, IDESC_QK);
           mma_commit(bars.s_full(0));
           if (n1 > 0) {
-            issue_qk(1, 0);
+            issue_qk(1, 0, 0, IDESC_QK);
             mma_commit(bars.s_full(1));
           }
           mma_commit(bars.k_empty(0));
@@ -247,7 +260,18 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!mbar_wait_sleep(bars.v_full(vs), ((j - 1) / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
           if (j < nkv && !mbar_wait_sleep(bars.k_full(ks), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) break;
           tc_fence_after();
-          for (int x = 0; x < 2; ++x) {
+          // S_x(j) for the keys whose score columns P does not use, as soon as
+          // the softmax has read S_x(j-1): it overlaps that softmax
+          for (int x = 0; ok && x < 2; ++x) {
+            if (j >= (x ? n1 : n0)) continue;
+            if (!mbar_wait_sleep(bars.s_free(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_qk(x, ks, P_COLS, IDESC_QK_TAIL);
+          }
+          for (int x = 0; ok && x < 2; ++x) {
             const int nx = x ? n1 : n0;
             if (j - 1 >= nx) continue;
             if (!mbar_wait_sleep(bars.p_full(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
@@ -257,7 +281,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             issue_pv(x, vs, j > 1);
             if (j < nx) {
-              issue_qk(x, ks);
+              // the keys over P's columns, once P V has read P (in order)
+              issue_qk(x, ks, 0, IDESC_QK_HEAD);
               mma_commit(bars.s_full(x));
             } else {
               mma_commit(bars.o_done(x));
@@ -296,6 +321,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     float l = 0.f;
     bool ok = n > 0;
     for (int j = 0; ok && j < n; ++j) {
+      // this tile's block scales, loaded while S is still being computed
+      const int kb0 = 2 * j;  // key blocks of this tile: 2j (keys 0-63) and 2j+1 (64-127)
+      const int kb1 = min(2 * j + 1, p.nblk - 1);
+      const float sk0 = sKs[kb0], sk1 = sKs[kb1], sv0 = sVs[kb0], sv1 = sVs[kb1];
       if (!__all_sync(0xffffffffu, mbar_wait(bars.s_full(x), j & 1, abort, p.status, SITE_S_FULL))) {
         ok = false;
         break;
@@ -313,12 +342,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[c][i]);
       }
-      const int kb0 = 2 * j;  // key blocks of this tile: 2j (keys 0-63) and 2j+1 (64-127)
-      const int kb1 = min(2 * j + 1, p.nblk - 1);
+      // S is in registers: the MMA warp may write the next S over the columns
+      // P will not use
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.s_free(x));
       // log2-domain score factor of each key half (folded into the FFMA
       // before the exponential); the max is taken on raw scores per half
-      const float f0 = crow * sKs[kb0], f1 = crow * sKs[kb1];
-      const float w0 = sVs[kb0] * wlift, w1 = sVs[kb1] * wlift;
+      const float f0 = crow * sk0, f1 = crow * sk1;
+      const float w0 = sv0 * wlift, w1 = sv1 * wlift;
       const int kv0 = j * BN;
       const bool edge = (kv0 + BN > p.N) || (CAUSAL && kv0 + BN - 1 > qt * BM);
       if (edge) {

@@ -7,6 +7,22 @@
 
 namespace fa {
 
+// Heads per group of the forward grid order: as many query heads as share
+// about 32 MiB of K and V (a quarter of L2), all of them when that covers
+// every head. Measured on B200 (forward, against heads fastest over all
+// heads): long128, 4 MiB of bf16 K/V per head, groups of 8: DRAM traffic
+// 608 -> 250 MB per launch, +3 %; gqa, groups of 32: +2 %; the FP8 workload,
+// groups of 8: 488 -> 154 MB, +3 %; gpt2 causal (0.5 MiB per head, groups of
+// 64): -3 % (groups of 8 there: -7 %, the causal tail).
+inline int raster_heads_for(long long BH, int group, long long kv_bytes_per_kv_head) {
+  const long long budget = 32ll << 20;
+  const long long per_qhead = kv_bytes_per_kv_head / (group > 0 ? group : 1);
+  long long G = per_qhead > 0 ? budget / per_qhead : BH;
+  if (G < 1) G = 1;
+  if (G > BH) G = BH;
+  return static_cast<int>(G);
+}
+
 struct FwdParams {
   float* lse;        // [B*Hq, N]; packed batches: [Hq, T]
   int* status;       // device status word (bounded waits report here)
@@ -26,6 +42,7 @@ struct FwdParams {
   int group;         // Hq / Hkv
   int num_qtiles;    // ceil(N / 128)
   int num_pairs;     // ceil(num_qtiles / 2): one CTA per pair of query tiles
+  int raster_heads;  // heads per group of the grid order (raster_heads_for)
   float scale_log2;  // scale * log2(e)
 };
 
@@ -100,6 +117,7 @@ struct Fp8Params {
   int group;
   int num_qtiles;
   int num_pairs;
+  int raster_heads;        // heads per group of the grid order (raster_heads_for)
   float score_log2;        // scale * log2(e), divided by d when rotated
 };
 

@@ -325,12 +325,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int s = j % C::NS;
         if (!mbar_wait_sleep(bars.k_full(s), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) return false;
         tc_fence_after();
-        const uint32_t kb = base + C::OFF_K + s * C::TILE_BYTES;
+        const uint64_t da = smem_desc_sw128(sQ, 16, 1024);
+        const uint64_t db = smem_desc_sw128(base + C::OFF_K + s * C::TILE_BYTES, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
-          mma_mx_ss(tmem + C::COL_S + (j & 1) * 128, smem_desc_sw128(sQ + kk * 32, 16, 1024),
-                    smem_desc_sw128(kb + kk * 32, 16, 1024), idesc_mx(BM, BN, false, kk), tmem + C::COL_SFQ,
-                    tmem + C::COL_SFK + (j & 1) * 4, kk > 0 ? 1u : 0u);
+          mma_mx_ss(tmem + C::COL_S + (j & 1) * 128, desc_plus(da, kk * 32), desc_plus(db, kk * 32),
+                    idesc_mx(BM, BN, false, kk), tmem + C::COL_SFQ, tmem + C::COL_SFK + (j & 1) * 4, kk > 0 ? 1u : 0u);
         mma_commit(bars.s_full(j & 1));
         mma_commit(bars.k_empty(s));
         return true;
@@ -344,13 +344,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait_sleep(bars.v_full(s), (j / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
         if (!mbar_wait_sleep(bars.p_full(j & 1), (j >> 1) & 1, abort, p.status, SITE_P_FULL)) break;
         tc_fence_after();
-        const uint32_t vb = base + C::OFF_V + s * C::TILE_BYTES;
+        const uint64_t dv = smem_desc_sw128(base + C::OFF_V + s * C::TILE_BYTES, 16384, 1024);
         // O += P_j V_j: 32 keys per instruction (P: 8 columns of 4 e4m3; V:
         // four 8-row groups of the MN-major tile), key block kk's scale byte
 #pragma unroll
         for (int kk = 0; kk < BN / 32; ++kk)
-          mma_mx_ts(tmem + C::COL_O, tmem + C::COL_S + (j & 1) * 128 + kk * 8,
-                    smem_desc_sw128(vb + kk * 4096, 16384, 1024), idesc_mx(BM, D, true, kk),
+          mma_mx_ts(tmem + C::COL_O, tmem + C::COL_S + (j & 1) * 128 + kk * 8, desc_plus(dv, kk * 4096),
+                    idesc_mx(BM, D, true, kk),
                     tmem + C::COL_SFP + (j & 1) * 4, tmem + C::COL_SFV + (j & 1) * 4, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bars.v_empty(s));
         mma_commit(bars.pv_done());
