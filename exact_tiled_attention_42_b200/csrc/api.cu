@@ -644,6 +644,7 @@ fa_status fa_fwd_mxfp8(const void* q, const void* k, const void* v, void* o, flo
   p.Hkv = Hkv;
   p.group = Hq / Hkv;
   p.num_qtiles = (N + 127) / 128;
+  p.raster_heads = fa::raster_heads_for(BH, Hq / Hkv, 2ll * N * d);  // e4m3 K and V
   p.score_log2 = scale * 1.4426950408889634f / (p.rotate ? static_cast<float>(d) : 1.0f);
   if (!p.status) return FA_ERR_CUDA;
   CUtensorMap tmQ, tmK, tmV, tmO;

@@ -100,9 +100,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // 1-D grid: heads fastest, the query tiles with the most key tiles (causal)
   // first, so the light tiles form the tail.
+  // heads in groups (raster_pairs, one query tile per CTA), heaviest tiles first
   const int BH = static_cast<int>(gridDim.x) / p.num_qtiles;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-  const int qt = p.num_qtiles - 1 - static_cast<int>(blockIdx.x) / BH;
+  int bh, qt;
+  raster_pairs(static_cast<int>(blockIdx.x), BH, p.num_qtiles, p.raster_heads, bh, qt);
   const int b = bh / p.Hq;
   const int hq = bh - b * p.Hq;
   int s0 = 0, n = p.N;

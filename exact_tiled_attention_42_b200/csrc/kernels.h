@@ -147,6 +147,7 @@ struct MxParams {
   int Hkv;
   int group;
   int num_qtiles;
+  int raster_heads;        // heads per group of the grid order (raster_heads_for)
   float score_log2;        // scale * log2(e), divided by d when rotated
 };
 
