@@ -133,12 +133,12 @@ size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 size_t up1024(size_t x) { return (x + 1023) & ~static_cast<size_t>(1023); }
 
 // 3-D map over an e4m3 [outer, N, d] tensor: 128 x 128 boxes, 128B swizzle.
-bool make_map_e4m3(CUtensorMap* m, const void* ptr, int d, int N, long long outer) {
+bool make_map_e4m3(CUtensorMap* m, const void* ptr, int d, int N, long long outer, int box_rows = 128) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(outer)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N) * d};
-  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -578,20 +578,22 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
 namespace {
 
 // MXFP8 workspace: e4m3 codes of Q, K, V, then the exponent bytes of Q, K
-// (4 per row) and V (nb32p per column), each region 1024-byte aligned.
+// (4 per row) and V (vexp_stride per column: a 4-byte word per 96-key tile),
+// each region 1024-byte aligned.
 struct MxLayout {
   size_t cq, ckv, eq, ekv, ev;
-  int nb32p;
+  int num_ktiles, vexp_stride;
 };
 MxLayout mx_layout(int B, int Hq, int Hkv, int N, int d) {
   MxLayout L;
-  L.nb32p = 4 * ((N + 127) / 128);
+  L.num_ktiles = (N + 95) / 96;
+  L.vexp_stride = 4 * L.num_ktiles;
   const size_t q = static_cast<size_t>(B) * Hq, kv = static_cast<size_t>(B) * Hkv;
   L.cq = up1024(q * N * d);
   L.ckv = up1024(kv * N * d);
   L.eq = up1024(q * N * 4);
   L.ekv = up1024(kv * N * 4);
-  L.ev = up1024(kv * d * L.nb32p);
+  L.ev = up1024(kv * d * L.vexp_stride);
   return L;
 }
 
@@ -639,17 +641,19 @@ fa_status fa_fwd_mxfp8(const void* q, const void* k, const void* v, void* o, flo
   p.lse = lse;
   p.status = status_ptr();
   p.N = N;
-  p.nb32p = L.nb32p;
+  p.num_ktiles = L.num_ktiles;
+  p.vexp_stride = L.vexp_stride;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.group = Hq / Hkv;
   p.num_qtiles = (N + 127) / 128;
+  p.num_pairs = (p.num_qtiles + 1) / 2;
   p.raster_heads = fa::raster_heads_for(BH, Hq / Hkv, 2ll * N * d);  // e4m3 K and V
   p.score_log2 = scale * 1.4426950408889634f / (p.rotate ? static_cast<float>(d) : 1.0f);
   if (!p.status) return FA_ERR_CUDA;
   CUtensorMap tmQ, tmK, tmV, tmO;
-  if (!make_map_e4m3(&tmQ, p.codes[0], d, N, BH) || !make_map_e4m3(&tmK, p.codes[1], d, N, BHkv) ||
-      !make_map_e4m3(&tmV, p.codes[2], d, N, BHkv) || !make_map_bf16(&tmO, o, d, N, BH, 128))
+  if (!make_map_e4m3(&tmQ, p.codes[0], d, N, BH) || !make_map_e4m3(&tmK, p.codes[1], d, N, BHkv, 96) ||
+      !make_map_e4m3(&tmV, p.codes[2], d, N, BHkv, 96) || !make_map_bf16(&tmO, o, d, N, BH, 128))
     return FA_ERR_CUDA;
   if (fa::launch_mxfp8_quant(p, stream) != cudaSuccess) return FA_ERR_CUDA;
   cudaError_t e = fa::launch_fwd_mxfp8(tmQ, tmK, tmV, tmO, p, static_cast<int>(BH), causal != 0, stream);

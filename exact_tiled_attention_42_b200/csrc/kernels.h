@@ -133,7 +133,8 @@ struct MxParams {
   const uint16_t* src[3];  // bf16 Q [B*Hq, N, d], K and V [B*Hkv, N, d]
   uint8_t* codes[3];       // e4m3 copies (Q and K rotated when rotate != 0), same layouts
   uint8_t* exps[3];        // E8M0 exponents (e + 127): Q [B*Hq, N, 4] and K [B*Hkv, N, 4] (one per
-                           // 32 columns), V [B*Hkv, d, nb32p] (one per 32 keys of a column)
+                           // 32 columns); V [B*Hkv, d, vexp_stride]: per column one 4-byte word per
+                           // 96-key tile, bytes 0-2 its three 32-key blocks, byte 3 zero
   int heads[3];            // B*Hq, B*Hkv, B*Hkv
   uint64_t rotation_seed;
   int rotate;
@@ -142,19 +143,22 @@ struct MxParams {
   float* lse;              // [B*Hq, N]
   int* status;
   int N;
-  int nb32p;               // 4 * ceil(N / 128): V's 32-key blocks per column, whole 128-key tiles
+  int num_ktiles;          // ceil(N / 96): the forward's key tiles
+  int vexp_stride;         // 4 * num_ktiles: bytes of V's exponents per column
   int Hq;
   int Hkv;
   int group;
   int num_qtiles;
+  int num_pairs;           // ceil(num_qtiles / 2): one CTA per pair of query tiles
   int raster_heads;        // heads per group of the grid order (raster_heads_for)
   float score_log2;        // scale * log2(e), divided by d when rotated
 };
 
 // MXFP8 pre-pass (rotation + MX quantisation of Q, K along d and of V along
-// the keys) and the MXFP8 forward (d = 128; one query tile per CTA, grid
-// BH * p.num_qtiles). tmQ8/tmK8/tmV8: e4m3 [B*H, N, d], 128 x 128 boxes, 128B
-// swizzle; tmO: bf16 output map as for the bf16 forward.
+// the keys) and the MXFP8 forward (d = 128; two query tiles per CTA, grid
+// BH * p.num_pairs). tmQ8: e4m3 [B*Hq, N, d], 128-row boxes; tmK8/tmV8: e4m3
+// [B*Hkv, N, d], 96-row boxes; 128B swizzle; tmO: bf16 output map as for the
+// bf16 forward.
 cudaError_t launch_mxfp8_quant(const MxParams& p, cudaStream_t stream);
 cudaError_t launch_fwd_mxfp8(const CUtensorMap& tmQ8, const CUtensorMap& tmK8, const CUtensorMap& tmV8,
                              const CUtensorMap& tmO, const MxParams& p, int BH, bool causal, cudaStream_t stream);

@@ -18,18 +18,25 @@
 // exceeds 1.75, so no element is clamped; rule "ocp" keeps the
 // specification's value and saturates at 448.
 //
-// Forward kernel: one 128-row query tile per CTA (tensor memory holds the
-// block scales next to two score buffers and O), 128-key tiles, the MMA order
-// S_0, S_1, PV_0, S_2, PV_1, ... of the wide-head kernel so the next Q K^T
-// overlaps the softmax. A row raises its running max only past TAU (log2
-// units; see TAU).
+// Forward kernel: the FP8 forward's layout (two 128-row query tiles per CTA,
+// a TMA producer warp, one MMA-issuing thread, two softmax warpgroups) on
+// 96-key tiles, three MX blocks each: tensor memory then holds both query
+// tiles' scores (96 columns, P over the first 24) and outputs (128) with 32
+// columns left for each tile's block-scale cells. The next tile's Q K^T is
+// issued in two parts: keys 32-95 as soon as the softmax has read S (s_free),
+// keys 0-31 (the columns P uses) after P V. A row raises its running max only
+// past TAU (log2 units; see TAU).
 // Block scales sit in tensor memory as the tensor cores read them: the scale
 // of A's row i (and block b along K) in lane i, column base + i/32, byte b;
 // the scale of B's column n in lane n % 32 of EVERY lane quarter (the tensor
 // cores read it from the quarter of the output row), column base + n/32.
+// Each softmax warpgroup writes its own tile's cells (Q once; K of tile j+1
+// before it signals s_free; V and P of tile j before p_full), so no cell is
+// shared by the two query tiles.
 //
-// Tensor memory: S_a [0,128), S_b [128,256), O [256,384), then scale cells:
-// Q [384,388), K x2 [388,396), V x2 [396,404), P x2 [404,412).
+// Tensor memory: S0 [0,96), S1 [96,192), O0 [192,320), O1 [320,448); scale
+// cells of query tile x from 448 + 32x: Q (4 columns), K (two slots of 4),
+// K for keys 32-95 (two slots of 4), V (two slots of 4), P (4).
 #include "common.cuh"
 #include "kernels.h"
 #include "rotation.cuh"
@@ -39,18 +46,25 @@ namespace {
 
 constexpr int D = 128;
 constexpr int BM = 128;
-constexpr int BN = 128;
-constexpr int PRODUCER_WARP = 4;
-constexpr int MMA_WARP = 5;
-constexpr int THREADS = 192;
+constexpr int BN = 96;  // key tile: three 32-key MX blocks
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
+// Three warpgroups: softmax of query tile 0 (warps 0-3) and 1 (warps 4-7);
+// warpgroup 2 holds the producer and MMA warps. After setup warpgroup 2 lowers
+// its registers so the softmax warps can rise (256 * 208 + 128 * 88 =
+// 384 * 168, checked against the compiled count before launching).
+constexpr int THREADS = 384;
+constexpr int REGS_SOFTMAX = 208;
+constexpr int REGS_OTHER = 88;
+static_assert(256 * REGS_SOFTMAX + 128 * REGS_OTHER <= THREADS * 168, "register split");
 // A row raises its running max only past TAU (log2 units). MX block scales
 // absorb any magnitude of P, so TAU bounds accuracy, not range: a stale max
 // leaves the row's largest term off the exact code 2^8 (P = 1) and, under the
 // specification's rule, open to the clamp at 448. Measured on the emulation
-// (N = 1000-2048, 0.1 % outliers): RMS error against exact attention within
-// 0.5 % (TAU = 2) / 2.2 % (TAU = 4) / 11 % (TAU = 8) of the one-tile
-// schedule; TAU = 4 rescales O in about a fifth of the key tiles of a
-// 4096-key row (TAU = 8: a twentieth, TAU = 0: four fifths).
+// (N = 1000-2048, 0.1 % outliers, 96-key tiles): RMS error against exact
+// attention within 0.6 % (TAU = 2) / 3.4 % (TAU = 4) / 11 % (TAU = 8) of the
+// one-tile schedule; TAU = 4 rescales O in about a fifth of the key tiles of
+// a 4096-key row (TAU = 8: a twentieth, TAU = 0: four fifths).
 constexpr float TAU = 4.0f;
 constexpr float LN2 = 0.69314718055994530942f;
 
@@ -78,7 +92,8 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 // One CTA per 64-row block of one (batch, head) of Q, K or V (grid z): 8 warps
 // x 8 rows, d/32 = 4 consecutive elements per lane. Q, K: the 8 lanes holding
 // one 32-column block share its exponent (shuffles). V: a block is 32 keys of
-// one column: per-warp column maxima meet in shared memory.
+// one column: per-warp column maxima meet in shared memory; V's exponents are
+// stored one 4-byte word per 96-key tile and column (the forward's tiles).
 __global__ void __launch_bounds__(256) mxfp8_quant_kernel(const MxParams p) {
   constexpr int E = D / 32;
   const int t = blockIdx.z;  // 0 = Q, 1 = K, 2 = V
@@ -144,7 +159,13 @@ __global__ void __launch_bounds__(256) mxfp8_quant_kernel(const MxParams p) {
       const float amax = fmaxf(fmaxf(colmax[w0][c], colmax[w0 + 1][c]), fmaxf(colmax[w0 + 2][c], colmax[w0 + 3][c]));
       const int ex = mx_exponent(amax, p.fit);
       inv[e] = pow2_neg(ex);
-      if ((warp & 3) == 0) p.exps[2][(static_cast<long long>(bh) * D + c) * p.nb32p + kb] = static_cast<uint8_t>(ex + 127);
+      // one 4-byte word per 96-key tile and column: bytes 0-2 the tile's three
+      // 32-key blocks, byte 3 zero
+      if ((warp & 3) == 0 && kb < 3 * p.num_ktiles) {
+        uint8_t* w = p.exps[2] + (static_cast<long long>(bh) * D + c) * p.vexp_stride + (kb / 3) * 4;
+        w[kb % 3] = static_cast<uint8_t>(ex + 127);
+        if (kb % 3 == 2) w[3] = 0;
+      }
     }
 #pragma unroll
     for (int rr = 0; rr < 8; ++rr) {
@@ -159,17 +180,29 @@ __global__ void __launch_bounds__(256) mxfp8_quant_kernel(const MxParams p) {
 
 // ------------------------------------------------------------------ forward
 struct Cfg {
-  static constexpr int TILE_BYTES = 128 * D;  // e4m3: 128 rows x 128 bytes
-  static constexpr int NS = 4;
+  static constexpr int Q_BYTES = BM * D;   // e4m3: 128 rows x 128 bytes
+  static constexpr int KV_BYTES = BN * D;  // 96 rows x 128 bytes
+  static constexpr int NS = 3;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = TILE_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
-  static constexpr int OFF_O = OFF_V + NS * TILE_BYTES;  // bf16 output staging, 32 KB
-  static constexpr int OFF_BAR = OFF_O + BM * D * 2;
-  static constexpr int NUM_BARS = 1 + 4 * NS + 2 + 2 + 5;
+  static constexpr int OFF_K = 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
+  static constexpr int OFF_O = OFF_V + NS * KV_BYTES;  // bf16 output staging, 2 x 32 KB
+  static constexpr int O_TILE_BYTES = BM * D * 2;
+  static constexpr int OFF_BAR = OFF_O + 2 * O_TILE_BYTES;
+  static constexpr int NUM_BARS = 1 + 4 * NS + 14;
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
-  static constexpr uint32_t COL_S = 0, COL_O = 256, COL_SFQ = 384, COL_SFK = 388, COL_SFV = 396, COL_SFP = 404;
+  // Tensor memory: scores of query tiles 0/1 (96 columns each, P over the
+  // first 24), outputs (128 each), then the block-scale cells of each query
+  // tile: Q (4 columns), K (two slots of 4: keys 0-31, 32-63, 64-95), K for
+  // the split-off keys 32-95 (two slots of 4: a scale address must sit on a
+  // 4-column boundary, so that part cannot start one column into K's slot),
+  // V (two slots of 4), P (4).
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 96, COL_O0 = 192, COL_O1 = 320;
+  static constexpr uint32_t COL_SF = 448, SF_PER_TILE = 32;
+  static constexpr uint32_t SF_Q = 0, SF_K = 4, SF_KT = 12, SF_V = 20, SF_P = 28;
   static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(COL_SF + 2 * SF_PER_TILE <= TMEM_COLS, "tensor memory budget");
+  static_assert(OFF_K % 1024 == 0 && KV_BYTES % 1024 == 0 && OFF_O % 1024 == 0, "128B-swizzle atoms");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -180,13 +213,15 @@ struct Bars {
   __device__ uint32_t k_empty(int s) const { return base + 8u * (1 + Cfg::NS + s); }
   __device__ uint32_t v_full(int s) const { return base + 8u * (1 + 2 * Cfg::NS + s); }
   __device__ uint32_t v_empty(int s) const { return base + 8u * (1 + 3 * Cfg::NS + s); }
-  __device__ uint32_t s_full(int b) const { return base + 8u * (1 + 4 * Cfg::NS + b); }
-  __device__ uint32_t p_full(int b) const { return base + 8u * (3 + 4 * Cfg::NS + b); }
-  __device__ uint32_t pv_done() const { return base + 8u * (5 + 4 * Cfg::NS); }
-  __device__ uint32_t o_final() const { return base + 8u * (6 + 4 * Cfg::NS); }
-  __device__ uint32_t epi() const { return base + 8u * (7 + 4 * Cfg::NS); }
-  __device__ uint32_t sf0_ready() const { return base + 8u * (8 + 4 * Cfg::NS); }
-  __device__ uint32_t teardown() const { return base + 8u * (9 + 4 * Cfg::NS); }
+  __device__ uint32_t s_full(int x) const { return base + 8u * (1 + 4 * Cfg::NS + x); }
+  __device__ uint32_t p_full(int x) const { return base + 8u * (3 + 4 * Cfg::NS + x); }
+  __device__ uint32_t o_done(int x) const { return base + 8u * (5 + 4 * Cfg::NS + x); }
+  __device__ uint32_t epi(int x) const { return base + 8u * (7 + 4 * Cfg::NS + x); }
+  // the softmax of query tile x has read S_x: the columns past P's may take the next S_x
+  __device__ uint32_t s_free(int x) const { return base + 8u * (9 + 4 * Cfg::NS + x); }
+  // query tile x's first scale cells (Q, K of tiles 0) are written
+  __device__ uint32_t sf_ready(int x) const { return base + 8u * (11 + 4 * Cfg::NS + x); }
+  __device__ uint32_t teardown() const { return base + 8u * (13 + 4 * Cfg::NS); }
 };
 
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -229,6 +264,11 @@ __device__ __forceinline__ void tmem_st_x4(uint32_t taddr, uint32_t a, uint32_t 
                "r"(d)
                : "memory");
 }
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
 
 template <bool CAUSAL>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -243,15 +283,20 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // heads in groups (raster_pairs, one query tile per CTA), heaviest tiles first
-  const int BH = static_cast<int>(gridDim.x) / p.num_qtiles;
-  int bh, qt;
-  raster_pairs(static_cast<int>(blockIdx.x), BH, p.num_qtiles, p.raster_heads, bh, qt);
+  // heads in groups (raster_pairs), the pairs of query tiles with the most
+  // key tiles first
+  const int BH = static_cast<int>(gridDim.x) / p.num_pairs;
+  int bh, pair;
+  raster_pairs(static_cast<int>(blockIdx.x), BH, p.num_pairs, p.raster_heads, bh, pair);
   const int b = bh / p.Hq;
   const int hq = bh - b * p.Hq;
   const int kvh = b * p.Hkv + hq / p.group;
-  const int kv_end = CAUSAL ? min((qt + 1) * BM, p.N) : p.N;
-  const int nkv = (kv_end + BN - 1) / BN;
+  const int qt0 = 2 * pair, qt1 = 2 * pair + 1;
+  const bool has1 = qt1 < p.num_qtiles;
+  auto ntiles = [&](int qt) { return ((CAUSAL ? min((qt + 1) * BM, p.N) : p.N) + BN - 1) / BN; };
+  const int n0 = ntiles(qt0);
+  const int n1 = has1 ? ntiles(qt1) : 0;
+  const int nkv = n0 > n1 ? n0 : n1;
 
   const Bars bars{base + C::OFF_BAR};
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::OFF_BAR + C::NUM_BARS * 8);
@@ -268,11 +313,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(bars.s_full(x), 1);
       mbar_init(bars.p_full(x), 4);
+      mbar_init(bars.o_done(x), 1);
+      mbar_init(bars.epi(x), 4);
+      mbar_init(bars.s_free(x), 4);
+      mbar_init(bars.sf_ready(x), 4);
     }
-    mbar_init(bars.pv_done(), 1);
-    mbar_init(bars.o_final(), 1);
-    mbar_init(bars.epi(), 4);
-    mbar_init(bars.sf0_ready(), 4);
     mbar_init(bars.teardown(), 1);
     *abort = 0;
     fence_barrier_init();
@@ -292,131 +337,197 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == PRODUCER_WARP) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bars.q_full(), C::TILE_BYTES);
-      tma_load_3d(base + C::OFF_Q, &tmQ, bars.q_full(), 0, qt * BM, bh);
-      int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % C::NS;
-        const uint32_t ph = (j / C::NS) & 1;
-        if (!mbar_wait_sleep(bars.k_empty(s), ph ^ 1, abort, p.status, SITE_K_EMPTY)) break;
-        mbar_arrive_expect_tx(bars.k_full(s), C::TILE_BYTES);
-        tma_load_3d(base + C::OFF_K + s * C::TILE_BYTES, &tmK, bars.k_full(s), 0, j * BN, kvh);
-        if (!mbar_wait_sleep(bars.v_empty(s), ph ^ 1, abort, p.status, SITE_V_EMPTY)) {
-          issued = 2 * j + 1;
-          break;
+  if (warp >= 8) {
+    setmaxnreg_dec<REGS_OTHER>();
+    if (warp == PRODUCER_WARP) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bars.q_full(), (has1 ? 2 : 1) * C::Q_BYTES);
+        tma_load_3d(base + C::OFF_Q, &tmQ, bars.q_full(), 0, qt0 * BM, bh);
+        if (has1) tma_load_3d(base + C::OFF_Q + C::Q_BYTES, &tmQ, bars.q_full(), 0, qt1 * BM, bh);
+        int issued = 0;
+        for (int j = 0; j < nkv; ++j) {
+          const int s = j % C::NS;
+          const uint32_t ph = (j / C::NS) & 1;
+          if (!mbar_wait_sleep(bars.k_empty(s), ph ^ 1, abort, p.status, SITE_K_EMPTY)) break;
+          mbar_arrive_expect_tx(bars.k_full(s), C::KV_BYTES);
+          tma_load_3d(base + C::OFF_K + s * C::KV_BYTES, &tmK, bars.k_full(s), 0, j * BN, kvh);
+          if (!mbar_wait_sleep(bars.v_empty(s), ph ^ 1, abort, p.status, SITE_V_EMPTY)) {
+            issued = 2 * j + 1;
+            break;
+          }
+          mbar_arrive_expect_tx(bars.v_full(s), C::KV_BYTES);
+          tma_load_3d(base + C::OFF_V + s * C::KV_BYTES, &tmV, bars.v_full(s), 0, j * BN, kvh);
+          issued = 2 * j + 2;
         }
-        mbar_arrive_expect_tx(bars.v_full(s), C::TILE_BYTES);
-        tma_load_3d(base + C::OFF_V + s * C::TILE_BYTES, &tmV, bars.v_full(s), 0, j * BN, kvh);
-        issued = 2 * j + 2;
-      }
-      if (*abort) {
-        drain_wait(bars.q_full(), 0);
-        for (int t = (issued > 2 * C::NS ? issued - 2 * C::NS : 0); t < issued; ++t) {
-          const int j = t >> 1;
-          drain_wait((t & 1) ? bars.v_full(j % C::NS) : bars.k_full(j % C::NS), (j / C::NS) & 1);
+        if (*abort) {
+          drain_wait(bars.q_full(), 0);
+          for (int t = (issued > 2 * C::NS ? issued - 2 * C::NS : 0); t < issued; ++t) {
+            const int j = t >> 1;
+            drain_wait((t & 1) ? bars.v_full(j % C::NS) : bars.k_full(j % C::NS), (j / C::NS) & 1);
+          }
         }
       }
-    }
-  } else if (warp == MMA_WARP) {
-    if (lane == 0) {
-      const uint32_t sQ = base + C::OFF_Q;
-      auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T (block scales of Q and K_j)
-        const int s = j % C::NS;
-        if (!mbar_wait_sleep(bars.k_full(s), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) return false;
-        tc_fence_after();
-        const uint64_t da = smem_desc_sw128(sQ, 16, 1024);
-        const uint64_t db = smem_desc_sw128(base + C::OFF_K + s * C::TILE_BYTES, 16, 1024);
+    } else if (warp == MMA_WARP) {
+      if (lane == 0) {
+        const uint32_t sQ = base + C::OFF_Q;
+        // S_x(j) over keys [key0, key0 + N) of the stage into their score
+        // columns; K's scale cells of tile j in slot j & 1 (keys 0-95, or the
+        // copy for keys 32-95)
+        auto issue_qk = [&](int x, int j, int key0, int N_) {
+          const int stage = j % C::NS;
+          const uint32_t sf = tmem + C::COL_SF + x * C::SF_PER_TILE;
+          const uint64_t da = smem_desc_sw128(sQ + x * C::Q_BYTES, 16, 1024);
+          const uint64_t db = smem_desc_sw128(base + C::OFF_K + stage * C::KV_BYTES + key0 * 128, 16, 1024);
+          const uint32_t sfb = sf + (key0 == 32 ? C::SF_KT : C::SF_K) + (j & 1) * 4;
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)
-          mma_mx_ss(tmem + C::COL_S + (j & 1) * 128, desc_plus(da, kk * 32), desc_plus(db, kk * 32),
-                    idesc_mx(BM, BN, false, kk), tmem + C::COL_SFQ, tmem + C::COL_SFK + (j & 1) * 4, kk > 0 ? 1u : 0u);
-        mma_commit(bars.s_full(j & 1));
-        mma_commit(bars.k_empty(s));
-        return true;
-      };
-      bool ok = mbar_wait_sleep(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&
-                mbar_wait_sleep(bars.sf0_ready(), 0, abort, p.status, SITE_P_FULL);
-      if (ok) ok = issue_s(0);
-      if (ok && nkv > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % C::NS;
-        if (!mbar_wait_sleep(bars.v_full(s), (j / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
-        if (!mbar_wait_sleep(bars.p_full(j & 1), (j >> 1) & 1, abort, p.status, SITE_P_FULL)) break;
-        tc_fence_after();
-        const uint64_t dv = smem_desc_sw128(base + C::OFF_V + s * C::TILE_BYTES, 16384, 1024);
-        // O += P_j V_j: 32 keys per instruction (P: 8 columns of 4 e4m3; V:
-        // four 8-row groups of the MN-major tile), key block kk's scale byte
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_mx_ss(tmem + (x ? C::COL_S1 : C::COL_S0) + key0, desc_plus(da, kk * 32), desc_plus(db, kk * 32),
+                      N_ == 32 ? idesc_mx(BM, 32, false, kk) : (N_ == 64 ? idesc_mx(BM, 64, false, kk) : idesc_mx(BM, BN, false, kk)),
+                      sf + C::SF_Q, sfb, kk > 0 ? 1u : 0u);
+        };
+        // O_x += P_x(j) V(j): 32 keys per instruction (P: 8 columns of four
+        // e4m3; V: four 8-row groups of the MN-major tile), key block kk's scale byte
+        auto issue_pv = [&](int x, int j, bool accumulate) {
+          const int stage = j % C::NS;
+          const uint32_t sf = tmem + C::COL_SF + x * C::SF_PER_TILE;
+          const uint64_t dv = smem_desc_sw128(base + C::OFF_V + stage * C::KV_BYTES, 16384, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BN / 32; ++kk)
-          mma_mx_ts(tmem + C::COL_O, tmem + C::COL_S + (j & 1) * 128 + kk * 8, desc_plus(dv, kk * 4096),
-                    idesc_mx(BM, D, true, kk),
-                    tmem + C::COL_SFP + (j & 1) * 4, tmem + C::COL_SFV + (j & 1) * 4, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bars.v_empty(s));
-        mma_commit(bars.pv_done());
-        if (j + 2 < nkv && !issue_s(j + 2)) break;
+          for (int kk = 0; kk < BN / 32; ++kk)
+            mma_mx_ts(tmem + (x ? C::COL_O1 : C::COL_O0), tmem + (x ? C::COL_S1 : C::COL_S0) + kk * 8,
+                      desc_plus(dv, kk * 4096), idesc_mx(BM, D, true, kk), sf + C::SF_P, sf + C::SF_V + (j & 1) * 4,
+                      (accumulate || kk > 0) ? 1u : 0u);
+        };
+        bool ok = mbar_wait_sleep(bars.q_full(), 0, abort, p.status, SITE_Q_FULL) &&
+                  mbar_wait_sleep(bars.k_full(0), 0, abort, p.status, SITE_K_FULL) &&
+                  mbar_wait_sleep(bars.sf_ready(0), 0, abort, p.status, SITE_P_FULL) &&
+                  (n1 == 0 || mbar_wait_sleep(bars.sf_ready(1), 0, abort, p.status, SITE_P_FULL));
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0, 0, BN);
+          mma_commit(bars.s_full(0));
+          if (n1 > 0) {
+            issue_qk(1, 0, 0, BN);
+            mma_commit(bars.s_full(1));
+          }
+          mma_commit(bars.k_empty(0));
+        }
+        for (int j = 1; ok && j <= nkv; ++j) {
+          const int vs = (j - 1) % C::NS;
+          const int ks = j % C::NS;
+          if (!mbar_wait_sleep(bars.v_full(vs), ((j - 1) / C::NS) & 1, abort, p.status, SITE_V_FULL)) break;
+          if (j < nkv && !mbar_wait_sleep(bars.k_full(ks), (j / C::NS) & 1, abort, p.status, SITE_K_FULL)) break;
+          tc_fence_after();
+          // S_x(j) for keys 32-95 (columns P does not use) once the softmax has
+          // read S_x(j-1) and written K's scales of tile j
+          for (int x = 0; ok && x < 2; ++x) {
+            if (j >= (x ? n1 : n0)) continue;
+            if (!mbar_wait_sleep(bars.s_free(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_qk(x, j, 32, BN - 32);
+          }
+          for (int x = 0; ok && x < 2; ++x) {
+            const int nx = x ? n1 : n0;
+            if (j - 1 >= nx) continue;
+            if (!mbar_wait_sleep(bars.p_full(x), (j - 1) & 1, abort, p.status, SITE_P_FULL)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(x, j - 1, j > 1);
+            if (j < nx) {
+              issue_qk(x, j, 0, 32);  // keys 0-31, over P's columns, after P V has read P
+              mma_commit(bars.s_full(x));
+            } else {
+              mma_commit(bars.o_done(x));
+            }
+          }
+          if (!ok) break;
+          if (j < nkv) mma_commit(bars.k_empty(ks));
+          mma_commit(bars.v_empty(vs));
+        }
       }
-      mma_commit(bars.o_final());
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 0-3)
-    const int row = warp * 32 + lane;
+    // ------------------------------------------------------------ softmax (warpgroups 0 and 1)
+    setmaxnreg_inc<REGS_SOFTMAX>();
+    const int x = warp >> 2;
+    const int qt = x ? qt1 : qt0;
+    const int n = x ? n1 : n0;
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
     const int qrow = qt * BM + row;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tO = tmem + lane_off + C::COL_O;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (x ? C::COL_S1 : C::COL_S0);
+    const uint32_t tO = tmem + lane_off + (x ? C::COL_O1 : C::COL_O0);
+    const uint32_t tSF = tmem + lane_off + C::COL_SF + x * C::SF_PER_TILE;
     const float cl2 = p.score_log2;
     const uint32_t* kexp = reinterpret_cast<const uint32_t*>(p.exps[1]) + static_cast<long long>(kvh) * p.N;
-    const uint32_t* vexp = reinterpret_cast<const uint32_t*>(p.exps[2]) + static_cast<long long>(kvh) * D * (p.nb32p / 4);
-    // Scale cells of B (K_j, V_j): column n in lane n % 32 of every quarter;
-    // this warp writes its quarter, lane r the columns r, 32 + r, 64 + r, 96 + r.
+    const uint32_t* vexp = reinterpret_cast<const uint32_t*>(p.exps[2]) + static_cast<long long>(kvh) * D * (p.vexp_stride / 4);
+    // K's scale cells of tile j (slot j & 1): key n of the tile in lane n % 32
+    // of every lane quarter, column n / 32, and the same for keys 32-95 alone
+    // (the split-off part of the next S); this warp writes its quarter
     auto write_k_scales = [&](int j) {
-      uint32_t c[4];
+      uint32_t c[3];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 3; ++q) {
         const int key = j * BN + 32 * q + lane;
         c[q] = key < p.N ? kexp[key] : 0u;
       }
-      tmem_st_x4(tmem + lane_off + C::COL_SFK + (j & 1) * 4, c[0], c[1], c[2], c[3]);
+      tmem_st_x4(tSF + C::SF_K + (j & 1) * 4, c[0], c[1], c[2], 0u);
+      tmem_st_x4(tSF + C::SF_KT + (j & 1) * 4, c[1], c[2], 0u, 0u);
     };
+    // V's scale cells of tile j (slot j & 1): column d in lane d % 32 of every
+    // quarter, column d / 32; bytes 0-2 the tile's three key blocks
     auto write_v_scales = [&](int j) {
       uint32_t c[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) c[q] = vexp[(32 * q + lane) * (p.nb32p / 4) + j];
-      tmem_st_x4(tmem + lane_off + C::COL_SFV + (j & 1) * 4, c[0], c[1], c[2], c[3]);
+      for (int q = 0; q < 4; ++q) c[q] = vexp[(32 * q + lane) * (p.vexp_stride / 4) + j];
+      tmem_st_x4(tSF + C::SF_V + (j & 1) * 4, c[0], c[1], c[2], c[3]);
     };
-    // Q's scale cell: row i in lane i, column COL_SFQ + i / 32
-    tmem_st_x1(tmem + lane_off + C::COL_SFQ + warp,
-               qrow < p.N ? reinterpret_cast<const uint32_t*>(p.exps[0])[static_cast<long long>(bh) * p.N + qrow] : 0u);
-    write_k_scales(0);
-    if (nkv > 1) write_k_scales(1);
-    tmem_wait_st();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bars.sf0_ready());
+    if (n > 0) {
+      // Q's scale cell: row i in lane i, column i / 32
+      tmem_st_x1(tSF + C::SF_Q + wq,
+                 qrow < p.N ? reinterpret_cast<const uint32_t*>(p.exps[0])[static_cast<long long>(bh) * p.N + qrow] : 0u);
+      write_k_scales(0);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.sf_ready(x));
+    }
 
-    float m = -INFINITY;  // running max of c s, as m + mlo (mlo: the rounding residual of m)
+    float m = -INFINITY;  // running max of c s, as m + mlo (mlo: m's rounding residual)
     float mlo = 0.f;
     float l = 0.f;
-    bool ok = nkv > 0;
-    for (int j = 0; ok && j < nkv; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bars.s_full(j & 1), (j >> 1) & 1, abort, p.status, SITE_S_FULL))) {
+    bool ok = n > 0;
+    for (int j = 0; ok && j < n; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bars.s_full(x), j & 1, abort, p.status, SITE_S_FULL))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t tS = tmem + lane_off + C::COL_S + (j & 1) * 128;
       float s[BN];
       {
-        uint32_t r[4][32];
+        uint32_t r[3][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_x32(tS + 32 * c, r[c]);
+        for (int c = 0; c < 3; ++c) tmem_ld_x32(tS + 32 * c, r[c]);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 3; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[c][i]);
       }
+      // S is in registers and tile j+1's K scales go into the slot S_x(j-1)
+      // used: the MMA warp may start the next S_x
+      if (j + 1 < n) {
+        write_k_scales(j + 1);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.s_free(x));
       const int kv0 = j * BN;
       if (kv0 + BN > p.N || (CAUSAL && kv0 + BN - 1 > qt * BM)) {
         const int lim = CAUSAL ? min(qrow + 1, p.N) : p.N;
@@ -433,18 +544,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
         const bool raise = tile_max > m + TAU;
         if (__any_sync(0xffffffffu, raise)) {
+          // O_x is stable: S_x(j) completed after P_x(j-1) V(j-1)
           const float m_new = raise ? tile_max : m;
           const float mlo_new = raise ? tile_lo : mlo;
           const float alpha = ex2((m - m_new) + (mlo - mlo_new));
           l *= alpha;
           m = m_new;
           mlo = mlo_new;
-          // O may still be receiving P_{j-1} V_{j-1}
-          if (!__all_sync(0xffffffffu, mbar_wait(bars.pv_done(), (j - 1) & 1, abort, p.status, SITE_O_DONE))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D; c += 16) {
             uint32_t r[16];
@@ -456,50 +562,50 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      // P = 2^(c s - m) in fp32; its MX blocks of 32 keys: exponent from the
+      // P = 2^(c s - m) in fp32, x = fl(fma(s, c, -m) - mlo) (exactly 0 at the
+      // key that set the max); its MX blocks of 32 keys: exponent from the
       // block's largest P, codes e4m3(P 2^-e)
-      // x = fl(fma(s, c, -m) - mlo): the fused product-minus-max is exact at
-      // the key that set the max (it equals mlo there), so that key gets x = 0
-      // and P = 1 exactly whatever the compiler fuses (its block's exponent
-      // and code must not depend on a product's rounding residual)
       const float nm = (m == -INFINITY) ? 0.f : -m;
       const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(nm, nm), nlo2 = make_float2(-mlo, -mlo);
       float2 lsum = make_float2(0.f, 0.f);
-      uint32_t pk[32];
+      uint32_t pk[24];
       uint32_t pexp = 0;
 #pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
+      for (int blk = 0; blk < 3; ++blk) {
         float pv[32];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float2 x = __fadd2_rn(__ffma2_rn(make_float2(s[32 * blk + 2 * i], s[32 * blk + 2 * i + 1]), c2, nm2), nlo2);
-          pv[2 * i] = ex2(x.x);
-          pv[2 * i + 1] = ex2(x.y);
+          const float2 xx = __fadd2_rn(__ffma2_rn(make_float2(s[32 * blk + 2 * i], s[32 * blk + 2 * i + 1]), c2, nm2), nlo2);
+          pv[2 * i] = ex2(xx.x);
+          pv[2 * i + 1] = ex2(xx.y);
           lsum = __fadd2_rn(lsum, make_float2(pv[2 * i], pv[2 * i + 1]));
         }
         const int ex = mx_exponent(row_max<32>(pv), p.fit);
-        const float inv = pow2_neg(ex);
+        const float inv = pow2_neg(ex);  // a power of two: P 2^-e is exact
+        const float2 inv2 = make_float2(inv, inv);
         pexp |= static_cast<uint32_t>(ex + 127) << (8 * blk);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          pk[8 * blk + i] = e4m3x4(__fmul_rn(pv[4 * i], inv), __fmul_rn(pv[4 * i + 1], inv),
-                                   __fmul_rn(pv[4 * i + 2], inv), __fmul_rn(pv[4 * i + 3], inv));
+        for (int i = 0; i < 8; ++i) {
+          const float2 a = __fmul2_rn(make_float2(pv[4 * i], pv[4 * i + 1]), inv2);
+          const float2 c = __fmul2_rn(make_float2(pv[4 * i + 2], pv[4 * i + 3]), inv2);
+          pk[8 * blk + i] = e4m3x4(a.x, a.y, c.x, c.y);
+        }
       }
       l += lsum.x + lsum.y;
-      tmem_st_x32(tS, pk);
-      tmem_st_x1(tmem + lane_off + C::COL_SFP + (j & 1) * 4 + warp, pexp);
+      tmem_st_x16(tS, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+      tmem_st_x8(tS + 16, pk + 16);
+      tmem_st_x1(tSF + C::SF_P + wq, pexp);
       write_v_scales(j);
-      if (j + 2 < nkv) write_k_scales(j + 2);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars.p_full(j & 1));
+      if (lane == 0) mbar_arrive(bars.p_full(x));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_sleep(bars.o_final(), 0, abort, p.status, SITE_O_DONE));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bars.o_done(x), 0, abort, p.status, SITE_O_DONE));
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.0f / l;
-      const uint32_t stage = base + C::OFF_O;
+      const uint32_t stage = base + C::OFF_O + x * C::O_TILE_BYTES;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t r[32];
@@ -519,8 +625,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars.epi());
-      if (row == 0 && mbar_wait_sleep(bars.epi(), 0, abort, p.status, SITE_O_DONE)) {
+      if (lane == 0) mbar_arrive(bars.epi(x));
+      if (row == 0 && mbar_wait(bars.epi(x), 0, abort, p.status, SITE_O_DONE)) {
         tma_store_3d(&tmO, stage, 0, qt * BM, bh);
         tma_store_3d(&tmO, stage + BM * 128, 64, qt * BM, bh);
         bulk_commit();
@@ -549,9 +655,19 @@ template <bool CAUSAL>
 cudaError_t launch_fwd(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmO,
                        const MxParams& p, int BH, cudaStream_t stream) {
   auto kern = fwd_mxfp8_kernel<CAUSAL>;
+  // The softmax warpgroups' setmaxnreg.inc waits until the CTA's register
+  // pool has room; make sure the compiled launch allocation covers the split.
+  static int regs = 0;
+  if (regs == 0) {
+    cudaFuncAttributes attr;
+    cudaError_t ea = cudaFuncGetAttributes(&attr, kern);
+    if (ea != cudaSuccess) return ea;
+    regs = attr.numRegs;
+  }
+  if (256 * REGS_SOFTMAX + 128 * REGS_OTHER > THREADS * regs) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(BH * p.num_qtiles), THREADS, Cfg::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmO, p);
+  kern<<<dim3(BH * p.num_pairs), THREADS, Cfg::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmO, p);
   return cudaGetLastError();
 }
 
@@ -559,7 +675,7 @@ cudaError_t launch_fwd(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUt
 
 cudaError_t launch_mxfp8_quant(const MxParams& p, cudaStream_t stream) {
   const int maxh = p.heads[0] > p.heads[1] ? p.heads[0] : p.heads[1];
-  dim3 grid(p.nb32p / 2, maxh, 3);  // 64-row blocks covering every 128-key tile
+  dim3 grid((3 * p.num_ktiles + 1) / 2, maxh, 3);  // 64-row blocks covering every 96-key tile
   mxfp8_quant_kernel<<<grid, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }

@@ -239,7 +239,7 @@ size_t fa_mxfp8_workspace_size(int B, int Hq, int Hkv, int N, int d);
  *   Q and K (after the rotation diag(sigma) H_d when use_rotation != 0, as in
  *   fa_fwd_fp8): each row in blocks of 32 columns;
  *   V: each column in blocks of 32 keys;
- *   P: each row of each 128-key tile in blocks of 32 keys.
+ *   P: each row of each 96-key tile in blocks of 32 keys.
  * Shared exponent e = floor(log2 amax) - 8 clamped to [-127, 127] (-127 for
  * a zero block), codes e4m3(x 2^-e) with saturation at 448 (scale_rule 0,
  * the specification's); scale_rule 1 takes e + 1 where amax's significand
@@ -252,8 +252,9 @@ size_t fa_mxfp8_workspace_size(int B, int Hq, int Hkv, int N, int d);
  * holds, each region starting on a 1024-byte boundary: e4m3 codes of Q
  * [B*Hq, N, d], K and V [B*Hkv, N, d]; exponent bytes (e + 127) of Q
  * [B*Hq, N, 4] and K [B*Hkv, N, 4] (one per 32 columns), and of V
- * [B*Hkv, d, nb] with nb = 4 * ceil(N / 128) (one per 32 keys of a column;
- * blocks past N hold the exponent of zeros, 0).
+ * [B*Hkv, d, nb] with nb = 4 * ceil(N / 96): per column one 4-byte word per
+ * 96-key tile (the forward's key tile), bytes 0-2 the exponents of its three
+ * 32-key blocks (blocks past N: the exponent of zeros, 0), byte 3 zero.
  */
 fa_status fa_fwd_mxfp8(const void* q, const void* k, const void* v, void* o, float* lse,
                        uint64_t rotation_seed, int use_rotation, int scale_rule,

@@ -157,9 +157,9 @@ def test_fp8_rejects_bad_arguments(lib):
 
 def test_mxfp8_rejects_bad_arguments(lib):
     ws = lib.fa_mxfp8_workspace_size(1, 2, 2, 300, 128)
-    # codes 2*300*128 each (three regions), exponents Q and K 2*300*4 each, V 2*128*12
+    # codes 2*300*128 each (three regions), exponents Q and K 2*300*4 each, V 2*128*(4 per 96-key tile)
     up = lambda x: (x + 1023) // 1024 * 1024
-    assert ws == 3 * up(2 * 300 * 128) + 2 * up(2 * 300 * 4) + up(2 * 128 * 12)
+    assert ws == 3 * up(2 * 300 * 128) + 2 * up(2 * 300 * 4) + up(2 * 128 * 4 * 4)
     assert lib.fa_mxfp8_workspace_size(1, 2, 2, 300, 64) == 0                 # d = 128 only
     def mx(q=P, rule=1, wsp=P, wsb=ws, Hq=2, d=128):
         return lib.fa_fwd_mxfp8(q, P, P, P, P, 7, 1, rule, wsp, wsb, 1, Hq, 2, 300, d, 0, 0.1, None)

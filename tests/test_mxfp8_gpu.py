@@ -3,11 +3,13 @@
 * The pre-pass is byte work decided in float32: its e4m3 codes and E8M0
   exponents must equal the oracle quantiser's (``oracle.mx_quantize``) bit for
   bit, for both scale rules, with and without the rotation; V's exponents are
-  per 32 keys of a column, blocks past N (up to a whole 128-key tile) hold the
+  per 32 keys of a column, stored one 4-byte word per 96-key tile (bytes 0-2
+  its blocks, byte 3 zero); blocks past N (up to a whole tile) hold the
   exponent of zeros.
 * The forward is compared with the oracle's fp64 emulation of the same steps
   (blocks of 32 along each contraction, P quantised per 32 keys of each
-  128-key tile, the running max raised only past 4 in log2 units). What may
+  96-key tile -- the kernel's key tile -- the running max raised only past 4
+  in log2 units). What may
   differ is what differs in the per-block FP8 path, with the same gates:
   bf16 rounding of O, fp32 scores and P against fp64, and hence the odd P
   code rounded to the neighbouring e4m3 value (at most 2^-3 P_ij |V_jc| per
@@ -34,6 +36,7 @@ from test_fp8_gpu import check_against_emulation
 pytestmark = pytest.mark.gpu
 
 TAU = 4.0   # the kernel's deferred-max threshold (log2 units)
+TILE = 96   # the kernel's key tile
 
 
 def up1024(x):
@@ -54,8 +57,9 @@ def run_mx(dev, causal, seed, rotate, rule):
 
 def split_workspace(ws, B, Hq, Hkv, N, d):
     """The documented layout: codes Q, K, V; exponent bytes Q [BHq, N, 4],
-    K [BHkv, N, 4], V [BHkv, d, nb]; each region 1024-byte aligned."""
-    nb = 4 * (-(-N // 128))
+    K [BHkv, N, 4], V [BHkv, d, nb] with nb = 4 ceil(N / 96); each region
+    1024-byte aligned."""
+    nb = 4 * (-(-N // TILE))
     sizes = [B * Hq * N * d, B * Hkv * N * d, B * Hkv * N * d, B * Hq * N * 4, B * Hkv * N * 4, B * Hkv * d * nb]
     out, off = [], 0
     for n in sizes:
@@ -90,9 +94,11 @@ def test_prepass_codes_and_exponents_bit_exact(rule, rotate, N):
         assert same.all(), f"{name}: {np.count_nonzero(~same)} codes differ"
         if name == "v":
             nb = e.shape[-2]                                # blocks of 32 keys: [B, H, nb, d]
-            got_e = exps[2]                                 # [B, H, d, nb_padded]
-            np.testing.assert_array_equal(got_e[..., :nb], np.swapaxes(e, -1, -2))
-            assert np.all(got_e[..., nb:] == -127)
+            words = exps[2].reshape(B, Hkv, d, -1, 4)       # [B, H, d, tiles, 4]
+            blocks = words[..., :3].reshape(B, Hkv, d, -1)  # the tiles' three blocks in order
+            np.testing.assert_array_equal(blocks[..., :nb], np.swapaxes(e, -1, -2))
+            assert np.all(blocks[..., nb:] == -127)
+            assert np.all(words[..., 3] == -127)            # byte 3 of each word is 0
         else:
             np.testing.assert_array_equal(exps[t], e)
 
@@ -108,7 +114,7 @@ def test_forward_matches_emulation(rule, causal, N, Hq, Hkv):
     o, lse, _ = run_mx(dev, causal, seed, True, rule)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
     o_emu, lse_emu = oracle.mxfp8_attention_forward(host["q"], host["k"], host["v"], causal, d ** -0.5, sigma,
-                                                    rule=rule, tau=TAU)
+                                                    tile=TILE, rule=rule, tau=TAU)
     check_against_emulation(o, lse, o_emu, lse_emu, host["q"], host["k"], host["v"], causal, d ** -0.5, sigma,
                             single_tile=lambda: oracle.mxfp8_attention_forward(
                                 host["q"], host["k"], host["v"], causal, d ** -0.5, sigma, tile=1 << 30,
@@ -120,7 +126,7 @@ def test_forward_without_rotation_matches_emulation():
     dev, host = make_inputs(1, 2, 2, 640, d, seed=171, outlier_rate=0.001, with_dout=False)
     o, lse, _ = run_mx(dev, False, 5, False, "fit")
     o_emu, lse_emu = oracle.mxfp8_attention_forward(host["q"], host["k"], host["v"], False, d ** -0.5, None,
-                                                    rule="fit", tau=TAU)
+                                                    tile=TILE, rule="fit", tau=TAU)
     check_against_emulation(o, lse, o_emu, lse_emu, host["q"], host["k"], host["v"], False, d ** -0.5, None,
                             single_tile=lambda: oracle.mxfp8_attention_forward(
                                 host["q"], host["k"], host["v"], False, d ** -0.5, None, tile=1 << 30,
