@@ -27,11 +27,12 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfa_b200.so")
-# Debug variant for the abort-path test: every bounded wait gives up after
-# 1 ms, and fa_debug_withhold_first_v() can keep the forward's first V tile
-# from being loaded. Never loaded by the product path.
+# Debug variant for the abort-path and bounds tests: every bounded wait gives
+# up after 1 ms, fa_debug_withhold_first_v() can keep the forward's first V
+# tile from being loaded, and every computed global index is checked against
+# its buffer (FA_ERR_BOUNDS). Never loaded by the product path.
 DEBUG_LIB = os.path.join(PKG, "libfa_b200_debug.so")
-DEBUG_FLAGS = ["-DFA_WAIT_TIMEOUT_NS=1000000ull", "-DFA_DEBUG_WITHHOLD"]
+DEBUG_FLAGS = ["-DFA_WAIT_TIMEOUT_NS=1000000ull", "-DFA_DEBUG_WITHHOLD", "-DFA_DEBUG_BOUNDS"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

@@ -141,8 +141,12 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p, long lo
   }
   const bool real = valid && n < len;
   const bool col = sub * 8 < p.d;
+  // elements of O, dO and the dQ accumulator; rows of the LSE vector
+  const long long elems = p.cu_seqlens ? static_cast<long long>(p.total) * p.Hq * p.d
+                                       : total_rows / p.Npad * p.N * p.d;
+  const long long lse_rows = p.cu_seqlens ? static_cast<long long>(p.total) * p.Hq : total_rows / p.Npad * p.N;
   float acc = 0.f;
-  if (real && col) {
+  if (real && col && in_bounds(tok * p.d + sub * 8 + 7, elems, p.status, 0)) {
     const long long off = tok * p.d + sub * 8;
     const uint4 ov = *reinterpret_cast<const uint4*>(p.o + off);
     const uint4 gv = *reinterpret_cast<const uint4*>(p.dout + off);
@@ -155,10 +159,10 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p, long lo
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   for (int off = lpr >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (valid && sub == 0) {
+  if (valid && sub == 0 && in_bounds(row, total_rows, p.status, 1)) {
     p.delta[row] = real ? acc : 0.f;
     const long long lse_i = p.cu_seqlens ? (bh - (bh / p.Hq) * p.Hq) * p.total + (tok / p.Hq) : bh * p.N + n;
-    p.neg_lse2[row] = real ? -p.lse[lse_i] * LOG2E : 0.f;
+    p.neg_lse2[row] = real && in_bounds(lse_i, lse_rows, p.status, 2) ? -p.lse[lse_i] * LOG2E : 0.f;
   }
 }
 
@@ -558,7 +562,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             for (int e = 0; e < 4; ++e)
               w4[e] = pack_bf16x2(__uint_as_float(t[q * 8 + 2 * e]) * mul, __uint_as_float(t[q * 8 + 2 * e + 1]) * mul);
             if (direct) {
-              if (j * BT + r < len && c + q * 8 < p.d)
+              if (j * BT + r < len && c + q * 8 < p.d &&
+                  in_bounds((grow - (which ? p.dv : p.dk)) + c + q * 8 + 7,
+                            static_cast<long long>(p.total) * p.Hkv * p.d, p.status, 3))
                 *reinterpret_cast<uint4*>(grow + c + q * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             } else {
               asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(box + sw128_offset(r, ((c & 63) >> 3) + q)),

@@ -29,6 +29,7 @@ enum WaitSite : int {
   SITE_S_FULL, SITE_P_FULL, SITE_O_DONE, SITE_TEARDOWN, SITE_LOAD_DRAIN,
   SITE_BWD = 32,
   SITE_SEQLENS = 64,  // a packed batch's offsets, checked on the device (FA_ERR_INVALID_ARG)
+  SITE_BOUNDS = 96,   // + the access: a computed global index outside its buffer (debug library)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -85,6 +86,23 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // Records the first error of a launch; later errors keep the first code.
 __device__ __forceinline__ void report_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
+}
+
+// Bounds check of a global index a kernel computes. In the debug library
+// (built with FA_DEBUG_BOUNDS) an index outside [0, limit) records
+// FA_ERR_BOUNDS | (SITE_BOUNDS + site) << 8 in the status word and the access
+// is skipped; the release library compiles the check away. (Tensor-memory and
+// shared-memory offsets are compile-time functions of the tile layouts, whose
+// budgets are static_asserts; the TMA copies are bounds-checked by hardware.)
+__device__ __forceinline__ bool in_bounds(long long idx, long long limit, int* status, int site) {
+#ifdef FA_DEBUG_BOUNDS
+  if (idx >= 0 && idx < limit) return true;
+  report_status(status, 7 | ((SITE_BOUNDS + site) << 8));
+  return false;
+#else
+  (void)idx, (void)limit, (void)status, (void)site;
+  return true;
+#endif
 }
 
 // Bounded wait for the phase with the given parity to complete. Returns false

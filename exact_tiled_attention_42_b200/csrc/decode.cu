@@ -333,6 +333,7 @@ __global__ void __launch_bounds__(THREADS, DecCfg<D>::MIN_CTAS)
             }
           }
         }
+        if (!in_bounds(slot * R + r, (p.ctas + p.units / p.tiles) * static_cast<long long>(R), p.status, 20)) continue;
         p.o_part[(slot * R + r) * D + col] = L > 0.f ? o / L : 0.f;
         if (col == 0) p.lse_part[slot * R + r] = L > 0.f ? (M + __log2f(L)) * LN2 : -INFINITY;
       }
@@ -363,6 +364,10 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const DecParams p, 
   const long long c_last = ((first_unit + p.tiles) * p.ctas - 1) / p.units;
   const int nparts = static_cast<int>(c_last - c_first + 1);
   const long long slot0 = c_first + bkv;
+  // every partial this row reads, and its output row, must lie in the buffers
+  if (!in_bounds(slot0 + nparts - 1, p.ctas + p.units / p.tiles, p.status, 21) ||
+      !in_bounds(static_cast<long long>(bh) * p.Nq + qi, p.units / p.tiles * p.group * p.Nq, p.status, 22))
+    return;
 
   float mx = -INFINITY;
   for (int j = lane; j < nparts; j += 32) mx = fmaxf(mx, p.lse_part[(slot0 + j) * p.R + r]);

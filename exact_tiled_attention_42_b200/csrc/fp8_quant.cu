@@ -72,12 +72,16 @@ __global__ void __launch_bounds__(256) fp8_quant_kernel(const Fp8Params p) {
 #pragma unroll
   for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
   const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
-  if (threadIdx.x == 0)
+  if (threadIdx.x == 0 && in_bounds(static_cast<long long>(bh) * p.nblk + blk, static_cast<long long>(p.heads[t]) * p.nblk,
+                                     p.status, 11))
     p.scales[t][static_cast<long long>(bh) * p.nblk + blk] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
     const int n = blk * 64 + warp * 8 + rr;
     if (n >= p.N) continue;
+    if (!in_bounds((static_cast<long long>(bh) * p.N + n) * D + lane * E + E - 1, static_cast<long long>(p.heads[t]) * p.N * D,
+                   p.status, 12))
+      continue;
     uint8_t* out = p.codes[t] + (static_cast<long long>(bh) * p.N + n) * D + lane * E;
     if (E == 4) {
       const uint32_t lo = e4m3x2(__fmul_rn(y[rr][0], inv), __fmul_rn(y[rr][1], inv));

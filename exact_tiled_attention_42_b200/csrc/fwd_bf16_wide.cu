@@ -342,7 +342,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int e = 0; e < 4; ++e)
             w[e] = pack_bf16x2(__uint_as_float(r[q * 8 + 2 * e]) * inv_l, __uint_as_float(r[q * 8 + 2 * e + 1]) * inv_l);
           if (direct) {
-            if (qrow < n)
+            if (qrow < n && in_bounds((static_cast<long long>(s0 + qrow) * p.Hq + hq) * D + c + q * 8 + 7,
+                                      static_cast<long long>(p.total) * p.Hq * D, p.status, 6))
               *reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(s0 + qrow) * p.Hq + hq) * D + c + q * 8) =
                   make_uint4(w[0], w[1], w[2], w[3]);
           } else {
@@ -368,10 +369,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       if (qrow < n) {
-        if (VARLEN)
-          p.lse[static_cast<size_t>(hq) * p.total + s0 + qrow] = (m + __log2f(l)) * LN2;
-        else
-          p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m + __log2f(l)) * LN2;
+        if (VARLEN) {
+          const long long li = static_cast<long long>(hq) * p.total + s0 + qrow;
+          if (in_bounds(li, static_cast<long long>(p.Hq) * p.total, p.status, 7)) p.lse[li] = (m + __log2f(l)) * LN2;
+        } else {
+          const long long li = static_cast<long long>(bh) * p.N + qrow;
+          if (in_bounds(li, static_cast<long long>(BH) * p.N, p.status, 7)) p.lse[li] = (m + __log2f(l)) * LN2;
+        }
       }
     }
   }

@@ -311,7 +311,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const float* sVs = p.scales[2] + static_cast<long long>(kvh) * p.nblk;
     // the head's largest V block scale (every lane computes it; L1-served)
     float vmax = 0.f;
-    for (int i = lane; i < p.nblk; i += 32) vmax = fmaxf(vmax, sVs[i]);
+    for (int i = lane; i < p.nblk; i += 32)
+      if (in_bounds(static_cast<long long>(kvh) * p.nblk + i, static_cast<long long>(p.heads[2]) * p.nblk, p.status, 8))
+        vmax = fmaxf(vmax, sVs[i]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
     const float wlift = P_LIFT / vmax;
@@ -324,7 +326,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       // this tile's block scales, loaded while S is still being computed
       const int kb0 = 2 * j;  // key blocks of this tile: 2j (keys 0-63) and 2j+1 (64-127)
       const int kb1 = min(2 * j + 1, p.nblk - 1);
-      const float sk0 = sKs[kb0], sk1 = sKs[kb1], sv0 = sVs[kb0], sv1 = sVs[kb1];
+      const bool kb_ok = in_bounds(static_cast<long long>(kvh) * p.nblk + kb1, static_cast<long long>(p.heads[1]) * p.nblk,
+                                   p.status, 9);
+      const float sk0 = kb_ok ? sKs[kb0] : 1.f, sk1 = kb_ok ? sKs[kb1] : 1.f;
+      const float sv0 = kb_ok ? sVs[kb0] : 1.f, sv1 = kb_ok ? sVs[kb1] : 1.f;
       if (!__all_sync(0xffffffffu, mbar_wait(bars.s_full(x), j & 1, abort, p.status, SITE_S_FULL))) {
         ok = false;
         break;
@@ -464,7 +469,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         bulk_commit();
         bulk_wait_read0();
       }
-      if (qrow < p.N) p.lse[static_cast<size_t>(bh) * p.N + qrow] = ((m + mlo) + __log2f(l)) * LN2;
+      if (qrow < p.N && in_bounds(static_cast<long long>(bh) * p.N + qrow, static_cast<long long>(p.heads[0]) * p.N,
+                                  p.status, 10))
+        p.lse[static_cast<size_t>(bh) * p.N + qrow] = ((m + mlo) + __log2f(l)) * LN2;
     }
   }
 

@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(256) mxfp8_quant_kernel(const MxParams p) {
       const int ex = mx_exponent(amax, p.fit);
       const float inv = pow2_neg(ex);
       const long long r = static_cast<long long>(bh) * p.N + n;
+      if (!in_bounds(r, static_cast<long long>(p.heads[t]) * p.N, p.status, 13)) continue;
       *reinterpret_cast<uint32_t*>(p.codes[t] + r * D + lane * E) =
           e4m3x4(__fmul_rn(y[rr][0], inv), __fmul_rn(y[rr][1], inv), __fmul_rn(y[rr][2], inv), __fmul_rn(y[rr][3], inv));
       if ((lane & 7) == 0) p.exps[t][r * 4 + (lane >> 3)] = static_cast<uint8_t>(ex + 127);
@@ -161,7 +162,9 @@ __global__ void __launch_bounds__(256) mxfp8_quant_kernel(const MxParams p) {
       inv[e] = pow2_neg(ex);
       // one 4-byte word per 96-key tile and column: bytes 0-2 the tile's three
       // 32-key blocks, byte 3 zero
-      if ((warp & 3) == 0 && kb < 3 * p.num_ktiles) {
+      if ((warp & 3) == 0 && kb < 3 * p.num_ktiles &&
+          in_bounds((static_cast<long long>(bh) * D + c) * p.vexp_stride + (kb / 3) * 4 + 3,
+                    static_cast<long long>(p.heads[2]) * D * p.vexp_stride, p.status, 14)) {
         uint8_t* w = p.exps[2] + (static_cast<long long>(bh) * D + c) * p.vexp_stride + (kb / 3) * 4;
         w[kb % 3] = static_cast<uint8_t>(ex + 127);
         if (kb % 3 == 2) w[3] = 0;
@@ -170,7 +173,8 @@ __global__ void __launch_bounds__(256) mxfp8_quant_kernel(const MxParams p) {
 #pragma unroll
     for (int rr = 0; rr < 8; ++rr) {
       const int n = blk * 64 + warp * 8 + rr;
-      if (n >= p.N) continue;
+      if (n >= p.N || !in_bounds(static_cast<long long>(bh) * p.N + n, static_cast<long long>(p.heads[2]) * p.N, p.status, 15))
+        continue;
       *reinterpret_cast<uint32_t*>(p.codes[2] + (static_cast<long long>(bh) * p.N + n) * D + lane * E) =
           e4m3x4(__fmul_rn(y[rr][0], inv[0]), __fmul_rn(y[rr][1], inv[1]), __fmul_rn(y[rr][2], inv[2]),
                  __fmul_rn(y[rr][3], inv[3]));
@@ -474,7 +478,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int q = 0; q < 3; ++q) {
         const int key = j * BN + 32 * q + lane;
-        c[q] = key < p.N ? kexp[key] : 0u;
+        c[q] = key < p.N && in_bounds(static_cast<long long>(kvh) * p.N + key, static_cast<long long>(p.heads[1]) * p.N,
+                                      p.status, 16)
+                   ? kexp[key]
+                   : 0u;
       }
       tmem_st_x4(tSF + C::SF_K + (j & 1) * 4, c[0], c[1], c[2], 0u);
       tmem_st_x4(tSF + C::SF_KT + (j & 1) * 4, c[1], c[2], 0u, 0u);
@@ -484,13 +491,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto write_v_scales = [&](int j) {
       uint32_t c[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) c[q] = vexp[(32 * q + lane) * (p.vexp_stride / 4) + j];
+      for (int q = 0; q < 4; ++q)
+        c[q] = in_bounds((static_cast<long long>(kvh) * D + 32 * q + lane) * (p.vexp_stride / 4) + j,
+                         static_cast<long long>(p.heads[2]) * D * (p.vexp_stride / 4), p.status, 17)
+                   ? vexp[(32 * q + lane) * (p.vexp_stride / 4) + j]
+                   : 0u;
       tmem_st_x4(tSF + C::SF_V + (j & 1) * 4, c[0], c[1], c[2], c[3]);
     };
     if (n > 0) {
       // Q's scale cell: row i in lane i, column i / 32
       tmem_st_x1(tSF + C::SF_Q + wq,
-                 qrow < p.N ? reinterpret_cast<const uint32_t*>(p.exps[0])[static_cast<long long>(bh) * p.N + qrow] : 0u);
+                 qrow < p.N && in_bounds(static_cast<long long>(bh) * p.N + qrow, static_cast<long long>(p.heads[0]) * p.N,
+                                         p.status, 18)
+                     ? reinterpret_cast<const uint32_t*>(p.exps[0])[static_cast<long long>(bh) * p.N + qrow]
+                     : 0u);
       write_k_scales(0);
       tmem_wait_st();
       tc_fence_before();
@@ -632,7 +646,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         bulk_commit();
         bulk_wait_read0();
       }
-      if (qrow < p.N) p.lse[static_cast<size_t>(bh) * p.N + qrow] = ((m + mlo) + __log2f(l)) * LN2;
+      if (qrow < p.N && in_bounds(static_cast<long long>(bh) * p.N + qrow, static_cast<long long>(p.heads[0]) * p.N,
+                                  p.status, 19))
+        p.lse[static_cast<size_t>(bh) * p.N + qrow] = ((m + mlo) + __log2f(l)) * LN2;
     }
   }
 

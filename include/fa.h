@@ -56,7 +56,8 @@ typedef enum {
   FA_ERR_MISALIGNED = 3,   /* a pointer that is not 16-byte aligned */
   FA_ERR_WORKSPACE = 4,    /* workspace pointer null or smaller than the *_workspace_size query */
   FA_ERR_CUDA = 5,         /* the CUDA runtime reported an error when launching */
-  FA_ERR_TIMEOUT = 6       /* a kernel gave up on a bounded wait (see fa_last_device_status) */
+  FA_ERR_TIMEOUT = 6,      /* a kernel gave up on a bounded wait (see fa_last_device_status) */
+  FA_ERR_BOUNDS = 7        /* debug library only: a kernel computed a global index outside its buffer */
 } fa_status;
 
 /*
