@@ -22,6 +22,9 @@ int main(void) {
   CHECK(fa_bwd_workspace_size(1, 2, 2, 128, 64) > 0);
   CHECK(fa_bwd_workspace_size(1, 3, 2, 128, 64) == 0);            /* Hq % Hkv != 0 */
   CHECK(fa_fp8_workspace_size(1, 2, 2, 256, 128) > 0);
+  CHECK(fa_mxfp8_workspace_size(1, 2, 2, 256, 128) > 0);
+  CHECK(fa_mxfp8_workspace_size(1, 2, 2, 256, 64) == 0);             /* d = 128 only */
+  CHECK(strcmp(fa_status_string(FA_ERR_BOUNDS), "FA_ERR_BOUNDS") == 0);
   CHECK(fa_decode_workspace_size(16, 32, 8, 1, 16384, 128, 0) > 0);
   CHECK(fa_decode_workspace_size(1, 8, 1, 4, 100, 128, 0) == 0);  /* 32 query rows per KV head */
   CHECK(fa_fwd(NULL, P, P, P, (float*)P, 1, 2, 2, 128, 64, 0, 0.125f, 0) == FA_ERR_INVALID_ARG);
