@@ -7,8 +7,9 @@ touching memory out of range (the stand-in for a device bounds checker,
 which is not available here). Every entry point runs through the debug
 library at small, odd sizes (ragged tiles, packed batches with an empty
 sequence, GQA, both masks): no check may fire, and the results must equal
-the release library's (bit for bit where the arithmetic order is fixed; dQ,
-summed by reduce-adds in whatever order they land, to 1e-6)."""
+the release library's (bit for bit where the arithmetic order is fixed; dQ
+is an fp32 sum of reduce-adds that land in any order, rounded to bf16, so
+the odd element may sit one bf16 step away: within 2^-7 relative)."""
 
 import numpy as np
 import pytest
@@ -65,7 +66,7 @@ def test_backward(dbg, N, d, causal):
     dev, _ = make_inputs(2, 4, 2, N, d, seed=3 * N + d, with_dout=True)
     o, lse = fa.fa_fwd(dev["q"], dev["k"], dev["v"], causal=causal)
     rel, out = both(dbg, lambda: fa.fa_bwd(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], causal=causal))
-    np.testing.assert_allclose(out[0], rel[0], rtol=1e-6, atol=1e-6)   # dQ
+    np.testing.assert_allclose(out[0], rel[0], rtol=2 ** -7, atol=1e-6)   # dQ: one bf16 step
     same(rel[1], out[1])                                               # dK
     same(rel[2], out[2])                                               # dV
 
@@ -85,7 +86,7 @@ def test_packed_batch(dbg, d):
     if d <= 128:
         o, lse = fa.fa_fwd_varlen(q, k, v, cu, max_seqlen=300, causal=True)
         rel, out = both(dbg, lambda: fa.fa_bwd_varlen(q, k, v, o, lse, do, cu, max_seqlen=300, causal=True))
-        np.testing.assert_allclose(out[0], rel[0], rtol=1e-6, atol=1e-6)
+        np.testing.assert_allclose(out[0], rel[0], rtol=2 ** -7, atol=1e-6)
         same(rel[1], out[1])
         same(rel[2], out[2])
 
