@@ -44,8 +44,10 @@ conversion rule (scale, clamp, zero block, where the two rules differ), the
 power-of-two scale and the range of each block's largest code, the element
 error bound, exact agreement with ``oracle.attention_forward`` when every
 operand is exactly representable and P is left unquantised, the error bound of
-P's quantisation otherwise, the blocking axis of V (a closed form with uniform
-P), and seeded comparisons with per-tensor FP8 and the 64-row-block FP8
+P's quantisation otherwise, the blocking axes of Q, K and V (closed forms), the
+E8M0 exponent range, a query row's independence of the other rows (P blocked
+along the keys of its own row), GQA against repeated KV heads, and seeded
+comparisons with per-tensor FP8 and the 64-row-block FP8
 emulation on inputs with outliers. ``tests/test_oracle_mxfp8_mutations.py``
 plants mistakes in a copy of this module and checks the pins catch them.
 """

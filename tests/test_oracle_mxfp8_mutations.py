@@ -37,6 +37,26 @@ MUTATIONS = [
     ("Q blocked along the query rows", "qh = mx_roundtrip(q.astype(np.float32), axis=-1, rule=rule)",
      "qh = mx_roundtrip(q.astype(np.float32), axis=-2, rule=rule)",
      [pins.test_q_is_blocked_along_d]),
+    ("P blocked along the query rows", "pq = mx_roundtrip(p, axis=-1, rule=rule)",
+     "pq = mx_roundtrip(p, axis=0, rule=rule)", [pins.test_each_query_row_depends_only_on_its_own_q]),
+    ("exponent not clamped to E8M0", "e = np.clip(e, E8M0_MIN, E8M0_MAX).astype(np.int64)", "e = e.astype(np.int64)",
+     [pins.test_exponent_clamped_to_the_e8m0_range]),
+    ("GQA head map", "kvh = h // g", "kvh = h % Hkv", [pins.test_gqa_equals_repeated_kv_heads]),
+    ("row sum of the quantised P",
+     "                l = l * alpha + p.sum(axis=1)\n                pq = mx_roundtrip(p, axis=-1, rule=rule) if quantize_p else p\n",
+     "                pq = mx_roundtrip(p, axis=-1, rule=rule) if quantize_p else p\n                l = l * alpha + pq.sum(axis=1)\n",
+     [pins.test_mxfp8_deferred_max_two_tile_closed_form]),
+    ("causal mask off by one", "s = np.where(np.arange(j0, j1)[None, :] > rows[:, None], -np.inf, s)",
+     "s = np.where(np.arange(j0, j1)[None, :] >= rows[:, None], -np.inf, s)",
+     [lambda: pins.test_exact_when_operands_representable_and_p_unquantised(True)]),
+    ("LSE left in log2", "lse[b, h] = (m + np.log2(l)) * math.log(2.0)", "lse[b, h] = (m + np.log2(l))",
+     [lambda: pins.test_exact_when_operands_representable_and_p_unquantised(False)]),
+    ("zero block given the exponent of its zero amax", "e = np.where(amax > 0, e, E8M0_MIN)", "e = e",
+     [pins.test_zero_block_and_ragged_tail]),
+    ("V rotated with Q and K", "    qh = mx_roundtrip(q.astype(np.float32), axis=-1, rule=rule)",
+     "    v = rotate_rows(v, sigma) / d if sigma is not None else v\n"
+     "    qh = mx_roundtrip(q.astype(np.float32), axis=-1, rule=rule)",
+     [lambda: pins.test_accuracy_on_the_fp8_input_recipe(21)]),
 ]
 
 

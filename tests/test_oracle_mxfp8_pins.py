@@ -64,6 +64,21 @@ def test_zero_block_and_ragged_tail():
     assert np.all(codes[0] == 0) and codes[1, 33] == 256.0 and np.count_nonzero(codes) == 1
 
 
+def test_exponent_clamped_to_the_e8m0_range():
+    """E8M0 holds exponents -127..127. A block with amax 2^-130 (reachable from
+    bf16 subnormals) takes e = -127, not -138, and keeps its value as the
+    code 2^-3; a block with amax 2^140 takes e = 127 and its code saturates
+    at 448. Both rules (the significand is 1)."""
+    x = np.zeros((2, 32))
+    x[0, 0] = 2.0 ** -130
+    x[1, 0] = 2.0 ** 140
+    for rule in ("ocp", "fit"):
+        codes, e = mx.mx_quantize(x, rule=rule)
+        np.testing.assert_array_equal(e[:, 0], [-127, 127])
+        assert codes[0, 0] == 0.125 and codes[1, 0] == E4M3_MAX
+        assert mx.mx_dequantize(codes, e)[0, 0] == 2.0 ** -130
+
+
 def test_scales_are_powers_of_two_and_largest_code_in_range():
     """Per block the largest |code| lies in [256, 448]: 2^8 <= amax / 2^e <
     2^9, clamped at 448."""
@@ -179,6 +194,38 @@ def test_q_is_blocked_along_d():
     o, _ = mx.mxfp8_attention_forward(q, k, v, False, 0.5, quantize_p=False)
     o_ref, _ = oracle.attention_forward(q, k, v, False, 0.5)
     np.testing.assert_allclose(o[0, 0, 1:], o_ref[0, 0, 1:], atol=2e-7)
+
+
+def test_each_query_row_depends_only_on_its_own_q():
+    """Q is blocked along d and P along the keys of one row, so a row's
+    output does not depend on the other query rows: changing rows 1.. leaves
+    row 0 as it was. (P blocked along the query rows would take each key's
+    block exponent from 32 rows' probabilities and move row 0 with them.)"""
+    rng = _rng(31)
+    q, k, v = (rng.standard_normal((1, 1, 64, 64)) for _ in range(3))
+    q2 = q.copy()
+    q2[0, 0, 1:] = 4.0 * rng.standard_normal((63, 64))
+    for rule in ("ocp", "fit"):
+        o1, l1 = mx.mxfp8_attention_forward(q, k, v, False, 0.125, rule=rule)
+        o2, l2 = mx.mxfp8_attention_forward(q2, k, v, False, 0.125, rule=rule)
+        np.testing.assert_allclose(o2[0, 0, 0], o1[0, 0, 0], rtol=0, atol=1e-12)
+        assert abs(l2[0, 0, 0] - l1[0, 0, 0]) <= 1e-12
+        assert np.max(np.abs(o2[0, 0, 1:] - o1[0, 0, 1:])) > 1e-3
+
+
+def test_gqa_equals_repeated_kv_heads():
+    """Query head h reads KV head h // (Hq / Hkv): four query heads over two KV
+    heads give what four KV heads 0, 0, 1, 1 give (the quantised copies of a
+    KV head are the same whichever query head reads them)."""
+    rng = _rng(32)
+    q = rng.standard_normal((1, 4, 96, 64))
+    k, v = (rng.standard_normal((1, 2, 96, 64)) for _ in range(2))
+    rep = lambda t: np.repeat(t, 2, axis=1)
+    for causal in (False, True):
+        o, lse = mx.mxfp8_attention_forward(q, k, v, causal, 0.125, rule="fit", tile=32, tau=4.0)
+        o2, lse2 = mx.mxfp8_attention_forward(q, rep(k), rep(v), causal, 0.125, rule="fit", tile=32, tau=4.0)
+        np.testing.assert_allclose(o, o2, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, lse2, rtol=0, atol=1e-12)
 
 
 @pytest.mark.parametrize("seed", [21, 22, 23])
