@@ -59,6 +59,21 @@ MUTATIONS = [
     ("per-tensor scale inverted", "s = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float64)",
      "s = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(1.0)).astype(np.float64)",
      [pins.test_per_tensor_quantize_closed_form]),
+    ("emulation: GQA head map", "            kvh = h // g\n            vref", "            kvh = h % Hkv\n            vref",
+     [lambda: pins.test_fp8_emulation_and_naive_gqa_equal_repeated_kv_heads(False)]),
+    ("naive: GQA head map", "s = scale * (qh[b, h, r0:r1] @ kh[b, h // g].T)",
+     "s = scale * (qh[b, h, r0:r1] @ kh[b, h % kh.shape[1]].T)",
+     [lambda: pins.test_fp8_emulation_and_naive_gqa_equal_repeated_kv_heads(False)]),
+    ("emulation: causal mask off by one",
+     "s = np.where(np.arange(j0, j1)[None, :] > np.arange(N)[:, None], -np.inf, s)",
+     "s = np.where(np.arange(j0, j1)[None, :] >= np.arange(N)[:, None], -np.inf, s)",
+     [lambda: pins.test_fp8_emulation_within_p_rounding_of_softmax_on_dequantised_operands(128, True, 0.0)]),
+    ("emulation: V's block weight not undone", "o[b, h] = acc * (vref / p_lift) / l[:, None]",
+     "o[b, h] = acc / p_lift / l[:, None]", [pins.test_fp8_deferred_max_two_tile_closed_form]),
+    ("e4m3 codes: exponent bias 8", "exp_field = np.where(normal, e + 7, 0)", "exp_field = np.where(normal, e + 8, 0)",
+     [pins.test_e4m3_codes_match_torch_bit_patterns]),
+    ("e4m3 rounding: no subnormal floor", "e = np.maximum(E - 1, _E4M3_MIN_NORMAL_EXP)", "e = E - 1",
+     [pins.test_e4m3_round_matches_torch_in_range]),
 ]
 
 SWAPPED = ("hadamard", "rotate_rows", "e4m3_round", "e4m3_encode", "e4m3_decode", "block_quantize",

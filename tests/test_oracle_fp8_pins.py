@@ -373,3 +373,23 @@ def test_fp8_deferred_max_two_tile_closed_form():
     o0, _ = oracle.fp8_attention_forward(q, k, v, False, scale, None, tile=1, tau=0.0)
     exact = (2 ** -0.5 * v[0, 0, 0] + v[0, 0, 1]) / (1 + 2 ** -0.5)
     np.testing.assert_allclose(o0[0, 0, 0], exact, rtol=1e-6, atol=1e-9)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_emulation_and_naive_gqa_equal_repeated_kv_heads(causal):
+    """Query head h reads KV head h // (Hq / Hkv) in both the emulation and
+    the naive baseline: four query heads over two KV heads give what four KV
+    heads 0, 0, 1, 1 give (a KV head's blocks, and the per-tensor amax, are the
+    same in both layouts)."""
+    rng = np.random.default_rng(61)
+    q = rng.standard_normal((1, 4, 150, 64))
+    k, v = (rng.standard_normal((1, 2, 150, 64)) for _ in range(2))
+    rep = lambda t: np.repeat(t, 2, axis=1)
+    sigma = sign_vector(9, 64)
+    o, lse = oracle.fp8_attention_forward(q, k, v, causal, 0.125, sigma)
+    o2, lse2 = oracle.fp8_attention_forward(q, rep(k), rep(v), causal, 0.125, sigma)
+    np.testing.assert_allclose(o, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse2, rtol=0, atol=1e-12)
+    n = oracle.naive_fp8_attention_forward(q, k, v, causal, 0.125)
+    n2 = oracle.naive_fp8_attention_forward(q, rep(k), rep(v), causal, 0.125)
+    np.testing.assert_allclose(n, n2, rtol=0, atol=1e-12)

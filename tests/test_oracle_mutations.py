@@ -34,6 +34,18 @@ MUTATIONS = [
      [lambda: pins.test_online_softmax_recurrence_is_exact(32, 0.0, False)]),
     ("LSE without max", "return e / l, (m + np.log(l))[:, 0]", "return e / l, (np.log(l))[:, 0]",
      [pins.test_lse_identity_without_max_shift]),
+    ("probabilities: GQA head map", "p[b, h], _ = _softmax_rows(_scores(q[b, h], k[b, h // g], scale, causal, 0, N))",
+     "p[b, h], _ = _softmax_rows(_scores(q[b, h], k[b, h % Hkv], scale, causal, 0, N))",
+     [lambda: pins.test_probabilities_times_v_is_the_forward_under_gqa(False)]),
+    ("decode alignment dropped", "i = np.arange(row0, row1)[:, None] + (kh.shape[0] - qh.shape[0])",
+     "i = np.arange(row0, row1)[:, None]", [lambda: pins.test_query_suffix_equals_rows_of_square_problem(True)]),
+    ("dK overwritten, not summed over the group", "dk[b, kv] += scale * (ds.T @ q[b, h, r0:r1])",
+     "dk[b, kv] = scale * (ds.T @ q[b, h, r0:r1])", [pins.test_gqa_equals_repeated_heads]),
+    ("dQ from P instead of dS", "dq[b, h, r0:r1] = scale * (ds @ kh)", "dq[b, h, r0:r1] = scale * (p @ kh)",
+     [lambda: pins.test_backward_matches_finite_differences(False, 2, 2)]),
+    ("row subset end off by one", "lo, hi = (0, N) if rows is None else rows\n    o = np.full",
+     "lo, hi = (0, N) if rows is None else (rows[0], rows[1] - 1)\n    o = np.full",
+     [pins.test_row_subset_matches_full_result]),
 ]
 
 

@@ -27,6 +27,16 @@ def test_probability_rows_sum_to_one(causal):
         assert np.all(np.triu(p[0, 0], 1) == 0)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_probabilities_times_v_is_the_forward_under_gqa(causal):
+    """P from attention_probabilities, multiplied by the V head each query head
+    reads (h // (Hq / Hkv)), is the forward's O."""
+    q, k, v = _rand((1, 4, 29, 16), 41), _rand((1, 2, 29, 16), 42), _rand((1, 2, 29, 16), 43)
+    p = oracle.attention_probabilities(q, k, causal, 0.25)
+    o, _ = oracle.attention_forward(q, k, v, causal, 0.25)
+    np.testing.assert_allclose(p @ np.repeat(v, 2, axis=1), o, atol=1e-13, rtol=0)
+
+
 # --- closed forms -----------------------------------------------------------
 
 @pytest.mark.parametrize("causal", [False, True])

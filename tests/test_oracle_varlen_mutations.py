@@ -36,6 +36,12 @@ MUTATIONS = [
      [lambda: pins.test_uniform_scores_average_within_the_sequence_only(False)]),
     ("dQ without the scale", "dq[s0:s1, h] = scale * (ds @ kh)", "dq[s0:s1, h] = ds @ kh",
      [pins.test_varlen_backward_finite_differences]),
+    ("decreasing offsets accepted", "np.any(np.diff(cu) < 0)", "False", [pins.test_bad_offsets_are_rejected]),
+    ("backward GQA head map", "            kv = h // g\n            qh, kh, vh, do", "            kv = h % Hkv\n            qh, kh, vh, do",
+     [lambda: pins.test_each_sequence_equals_the_fixed_length_oracle(True)]),
+    ("an empty sequence ends the batch", "        if n == 0:\n            continue\n        for h in range(Hq):\n            qh, kh",
+     "        if n == 0:\n            break\n        for h in range(Hq):\n            qh, kh",
+     [pins.test_other_sequences_do_not_move_the_result]),
 ]
 
 
