@@ -16,6 +16,17 @@ def test_splitmix64_is_counter_based_and_deterministic():
     assert not np.array_equal(a, splitmix64(43, np.arange(10, dtype=np.uint64)))
 
 
+def test_splitmix64_known_answers():
+    """Known-answer values of SplitMix64 (Steele, Lea and Flood 2014; the
+    reference C implementation's next()): the first outputs with the state
+    seeded to 1234567, and the first output from state 0 (0xE220A8397B1DCDAF).
+    Output i of the counter form is output i of the sequential generator."""
+    got = splitmix64(1234567, np.arange(5, dtype=np.uint64)).tolist()
+    assert got == [6457827717110365317, 3203168211198807973, 9817491932198370423, 4593380528125082431,
+                   16408922859458223821]
+    assert int(splitmix64(0, np.zeros(1, dtype=np.uint64))[0]) == 0xE220A8397B1DCDAF
+
+
 def test_normal_moments():
     x = normal(7, 0, 1 << 20)
     assert abs(x.mean()) < 5e-3
