@@ -186,8 +186,10 @@ size_t fa_fp8_workspace_size(int B, int Hq, int Hkv, int N, int d);
  * `rotation_seed` by SplitMix64, the same for Q and K) when use_rotation is
  * non-zero; Q, K, V are quantised with one float32 scale per 64-row block
  * (s = amax / 448); P is quantised per 128-key tile with V's block scale
- * folded in. Inputs are bf16; O is bf16, LSE float32. Only d = 128 is built
- * (FA_ERR_UNSUPPORTED otherwise). The workspace is overwritten; afterwards it
+ * folded in. Inputs are bf16; O is bf16, LSE float32. Only d = 128 is built,
+ * and B * Hq at most 65535 (FA_ERR_UNSUPPORTED otherwise; the same limits
+ * hold for fa_fp8_quantize and fa_fwd_fp8_quantized). The workspace is
+ * overwritten; afterwards it
  * holds, each region starting on a 1024-byte boundary: e4m3 codes of Q
  * [B*Hq, N, d], K and V [B*Hkv, N, d], then float32 block scales of Q
  * [B*Hq, ceil(N/64)], K and V [B*Hkv, ceil(N/64)].
@@ -245,8 +247,8 @@ size_t fa_mxfp8_workspace_size(int B, int Hq, int Hkv, int N, int d);
  * a zero block), codes e4m3(x 2^-e) with saturation at 448 (scale_rule 0,
  * the specification's); scale_rule 1 takes e + 1 where amax's significand
  * exceeds 1.75, so that no element saturates. Other scale_rule values:
- * FA_ERR_INVALID_ARG. Only d = 128 is built (FA_ERR_UNSUPPORTED otherwise);
- * B * Hq at most 65535. bf16 q [B, Hq, N, d], k, v [B, Hkv, N, d] and o
+ * FA_ERR_INVALID_ARG. Only d = 128 is built, and B * Hq at most 65535
+ * (FA_ERR_UNSUPPORTED otherwise). bf16 q [B, Hq, N, d], k, v [B, Hkv, N, d] and o
  * [B, Hq, N, d], float32 lse [B, Hq, N], all 16-byte aligned and owned by the
  * caller. The workspace (at least fa_mxfp8_workspace_size bytes, 16-byte
  * aligned, else FA_ERR_WORKSPACE / FA_ERR_MISALIGNED) is overwritten; it then

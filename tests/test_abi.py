@@ -174,6 +174,18 @@ def test_mxfp8_rejects_bad_arguments(lib):
     assert mx(Hq=3) == 1                                                      # Hq % Hkv
 
 
+def test_fp8_paths_reject_more_than_65535_query_heads(lib):
+    """The pre-passes put B * Hq on a grid dimension of at most 65535."""
+    for B, Hq in ((1, 65536), (2, 32768)):
+        ws8 = lib.fa_fp8_workspace_size(B, Hq, 1, 1, 128)
+        wsm = lib.fa_mxfp8_workspace_size(B, Hq, 1, 1, 128)
+        assert ws8 > 0 and wsm > 0
+        assert lib.fa_fwd_fp8(P, P, P, P, P, 7, 1, P, ws8, B, Hq, 1, 1, 128, 0, 0.1, None) == 2
+        assert lib.fa_fp8_quantize(P, P, P, 7, 1, P, ws8, B, Hq, 1, 1, 128, None) == 2
+        assert lib.fa_fwd_fp8_quantized(P, ws8, P, P, 1, B, Hq, 1, 1, 128, 0, 0.1, None) == 2
+        assert lib.fa_fwd_mxfp8(P, P, P, P, P, 7, 1, 1, P, wsm, B, Hq, 1, 1, 128, 0, 0.1, None) == 2
+
+
 def test_workspace_sizes_are_linear_in_n(lib):
     """The score matrix the pages size (4,096 tokens -> 16.7 million entries,
     128K -> 16.4 billion) is never stored: workspace grows linearly in N."""
