@@ -26,7 +26,9 @@
  *     bf16 tensors are passed as raw 16-bit storage.
  *   - d is 64, 96 or 128 (96 runs on the 128-column tiles with the extra
  *     columns zero-filled on load and clipped on store; its FLOP cost is
- *     that of 128); N >= 1; Hq is a multiple of Hkv; scale is finite and > 0.
+ *     that of 128); the bf16 forwards (fa_fwd, fa_fwd_varlen) also take 192
+ *     and 256; each entry point states its own set. N >= 1; Hq is a multiple
+ *     of Hkv; scale is finite and > 0.
  *   - Calls are asynchronous on `stream` (0 = legacy default stream), like a
  *     kernel launch; outputs are valid once the stream has been synchronised.
  *   - The caller owns every buffer, workspaces included. The library allocates
@@ -62,16 +64,19 @@ typedef enum {
 
 /*
  * Forward pass. Writes O (bf16, [B,Hq,N,d]) and LSE (float32, [B,Hq,N],
- * natural log). `lse` may not be null (the backward needs it).
+ * natural log). `lse` may not be null (the backward needs it). d is 64, 96,
+ * 128, 192 or 256 (FA_ERR_UNSUPPORTED otherwise); 192 and 256 run one
+ * 128-row query tile per CTA over 64-key tiles.
  */
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                  int B, int Hq, int Hkv, int N, int d, int causal, float scale,
                  cudaStream_t stream);
 
 /*
- * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) (float32,
- * [B,Hq,N]) and the float32 dQ accumulator ([B,Hq,N,d]), each rounded up to
- * 256 bytes. Linear in N. Returns 0 for invalid sizes.
+ * Bytes of device workspace fa_bwd needs: D = rowsum(dO * O) and
+ * -LSE * log2(e), each float32 [B*Hq, Npad] with Npad = 128 * ceil(N / 128),
+ * and the float32 dQ accumulator [B, Hq, N, d], each rounded up to 256
+ * bytes. Linear in N. Returns 0 for invalid sizes (fa_bwd's d: 64, 96, 128).
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
 
@@ -81,7 +86,8 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int N, int d);
  * dK = scale dS^T Q, with dK and dV summed over the Hq / Hkv query heads that
  * share a KV head. `o` and `lse` are fa_fwd's outputs for the same inputs.
  * dq, dk, dv (bf16) are overwritten, not accumulated. The workspace is
- * overwritten; its contents on entry do not matter.
+ * overwritten; its contents on entry do not matter. d is 64, 96 or 128
+ * (FA_ERR_UNSUPPORTED otherwise).
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                  const void* dout, void* dq, void* dk, void* dv,
@@ -108,7 +114,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * sequence longer than max_seqlen or offsets outside [0, T] make the kernels
  * skip that sequence and record FA_ERR_INVALID_ARG | (64 << 8) in the device
  * status word (fa_last_device_status). T = 0 or max_seqlen = 0 returns FA_OK
- * without launching. d is 64, 96 or 128.
+ * without launching. d is 64, 96, 128, 192 or 256 for fa_fwd_varlen and 64, 96
+ * or 128 for fa_bwd_varlen.
  */
 fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
                         int B, int Hq, int Hkv, int total, int max_seqlen, int d, int causal, float scale,
