@@ -316,9 +316,10 @@ const char* fa_status_string(fa_status s);
  * Device status word of the current device, then cleared. 0 when no kernel
  * has given up on a bounded wait or met bad packed-batch offsets since the
  * last call. Otherwise the low byte is an fa_status (FA_ERR_TIMEOUT, or
- * FA_ERR_INVALID_ARG for offsets) and bits 8.. name the wait that gave up
- * (64: the offsets check). Synchronises the device. Returns -1 if the word
- * could not be read.
+ * FA_ERR_INVALID_ARG for offsets; in the debug library also FA_ERR_BOUNDS)
+ * and bits 8.. name the site: the wait that gave up, 64 for the offsets
+ * check, 96 + n for bounds check n. Synchronises the device. Returns -1 if
+ * the word could not be read.
  */
 int fa_last_device_status(void);
 
