@@ -15,7 +15,9 @@ every step's inputs copied from pinned host memory and all results read back
 kernels); `fp8`, the FP8 workload's pre-pass + forward in TFLOP/s (and the
 MXFP8 forward on the same inputs); `decode`,
 one decode step (a query row per head against a 16K-key cache) in GB/s against
-the measured HBM copy bandwidth.
+the measured HBM copy bandwidth; `workloads`, the other bf16 workloads (GQA
+32/8 heads at N = 8192, d = 64 at N = 2048 causal and not, and the tiny
+N = 128 case in GB/s); `roofline`, the dominant kernel against its peak.
 
 Multi-GPU: every (batch, head) is an independent problem, so ranks run the
 same per-GPU workload with no collective on the data path (weak scaling); the
